@@ -1,0 +1,77 @@
+"""Sigmoid top-k router, fp64 reference.  TEST INFRASTRUCTURE ONLY.
+
+What the pages fix:
+  * "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, row
+    "Sigmoid router with Quantile Balancing": sigmoid scores pick 16 of 896
+    experts.  The same row appears in "Gemma 4 31B vs Kimi K3" (archdiff).
+  * "Kimi K3" (llm-atlas), raw config fields: moe_router_activation_func
+    sigmoid, num_experts 896, num_experts_per_token 16, moe_renormalize true,
+    routed_scaling_factor 1, use_grouped_topk true with num_expert_group 1 and
+    topk_group 1.  One group makes grouped top-k plain top-k.
+
+Readings (the pages leave these open):
+  R6 The bias is added to the logit, z = x.W_r + b, and both selection and
+     weights come from s = sigmoid(z).  The per-step Quantile Balancing rule is
+     unpublished, so b is an input.
+  R7 Selection is by z in descending order; on equal z the lower expert index
+     wins.  sigmoid is monotone, so this is selection by s in exact arithmetic,
+     and it avoids ties created by rounding s.
+  R8 Weights: w_j = s_j / sum of the selected s (renormalise, scale factor 1).
+     The output order is the selection order.
+  R9 The "16th/17th gap" of a token is sigmoid(z_(k)) - sigmoid(z_(k+1)) in fp64
+     (z_(i) is the i-th largest logit); it is +inf when k == E.
+"""
+import numpy as np
+
+
+def router_logits(x, W_r, bias=None):
+    """z[t, e] = sum_i x[t, i] * W_r[i, e] + b[e], in fp64 (R6).
+
+    x: [T, d] values (bf16 inputs are exact in fp64); W_r: [d, E]; bias: [E] or None.
+    """
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(W_r, dtype=np.float64)
+    if bias is not None:
+        z = z + np.asarray(bias, dtype=np.float64)[None, :]
+    return z
+
+
+def sigmoid(z):
+    z = np.asarray(z, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def topk_select(z, k):
+    """Indices of the k largest logits per row, descending, lower index on ties (R7).
+
+    z: [T, E] (any float type; compared exactly as fp64).
+    Returns int32 [T, k].
+    """
+    z = np.asarray(z, dtype=np.float64)
+    T, E = z.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    # lexsort sorts by the last key first: primary key -z (descending z), then index.
+    idx = np.empty((T, k), dtype=np.int32)
+    cols = np.arange(E)
+    for t in range(T):
+        order = np.lexsort((cols, -z[t]))
+        idx[t] = order[:k]
+    return idx
+
+
+def route(z, k):
+    """Selection, renormalised weights and the k/k+1 score gap (R7, R8, R9).
+
+    Returns (idx int32 [T,k], w fp64 [T,k], gap fp64 [T]).
+    """
+    z = np.asarray(z, dtype=np.float64)
+    T, E = z.shape
+    idx = topk_select(z, k)
+    s_sel = sigmoid(np.take_along_axis(z, idx.astype(np.int64), axis=1))
+    w = s_sel / np.sum(s_sel, axis=1, keepdims=True)
+    if k < E:
+        zs = -np.sort(-z, axis=1)
+        gap = sigmoid(zs[:, k - 1]) - sigmoid(zs[:, k])
+    else:
+        gap = np.full(T, np.inf)
+    return idx, w, gap

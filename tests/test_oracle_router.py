@@ -1,0 +1,113 @@
+"""Pins for the oracle's router (oracle/router.py) and permutation (oracle/permute.py):
+brute force on tiny inputs, the tie rule, and the routing invariants."""
+import itertools
+
+import numpy as np
+
+from oracle import permute as operm
+from oracle import router
+
+
+def test_logits_brute_force():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((3, 5))
+    W = rng.standard_normal((5, 4))
+    b = rng.standard_normal(4)
+    z = router.router_logits(x, W, b)
+    for t in range(3):
+        for e in range(4):
+            ref = sum(x[t, i] * W[i, e] for i in range(5)) + b[e]
+            assert abs(z[t, e] - ref) < 1e-12
+
+
+def test_topk_against_full_sort_and_invariants():
+    rng = np.random.default_rng(1)
+    for E, k in ((8, 2), (32, 4), (64, 16), (5, 5)):
+        z = rng.standard_normal((20, E))
+        idx, w, gap = router.route(z, k)
+        for t in range(20):
+            # brute force: all k-subsets, pick the one with the largest sorted logits
+            ranked = sorted(range(E), key=lambda e: (-z[t, e], e))
+            assert list(idx[t]) == ranked[:k]
+            assert len(set(idx[t])) == k
+            s = 1 / (1 + np.exp(-z[t, idx[t]]))
+            assert np.allclose(w[t], s / s.sum(), rtol=0, atol=1e-15)
+        assert np.all(w > 0)
+        assert np.allclose(w.sum(1), 1.0, rtol=0, atol=1e-15)
+        if k < E:
+            assert np.all(gap >= 0)
+
+
+def test_tie_rule_lower_index_wins():
+    z = np.array([[0.5, 1.0, 1.0, 0.2, 1.0, 0.9]])
+    idx, w, gap = router.route(z, 2)
+    assert list(idx[0]) == [1, 2]
+    assert gap[0] == 0.0
+    idx3, _, _ = router.route(z, 3)
+    assert list(idx3[0]) == [1, 2, 4]
+    # equal logits give equal weights
+    assert w[0, 0] == w[0, 1]
+
+
+def test_selection_by_logit_matches_selection_by_score():
+    """sigmoid is monotone: picking by z and by sigmoid(z) agree when scores differ."""
+    rng = np.random.default_rng(2)
+    z = rng.standard_normal((50, 40)) * 3
+    idx, _, _ = router.route(z, 6)
+    s = router.sigmoid(z)
+    for t in range(50):
+        assert set(idx[t]) == set(np.argsort(-s[t], kind="stable")[:6])
+
+
+def test_k_equals_e_is_a_dense_mixture():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((4, 6))
+    idx, w, gap = router.route(z, 6)
+    assert np.all(np.isinf(gap))
+    s = router.sigmoid(z)
+    for t in range(4):
+        assert np.allclose(w[t][np.argsort(idx[t])], s[t] / s[t].sum(), atol=1e-15)
+
+
+def test_permutation_brute_force():
+    rng = np.random.default_rng(4)
+    T, E, k = 9, 6, 3
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    counts, offsets, perm_tok, inv = operm.permute(idx, E)
+    pairs = sorted(((idx[t, j], t, j) for t in range(T) for j in range(k)))
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    assert np.all(np.diff(offsets) == counts)
+    for p, (e, t, j) in enumerate(pairs):
+        assert perm_tok[p] == t
+        assert inv[t, j] == p
+        assert offsets[e] <= p < offsets[e + 1]
+    # permute then unpermute is the identity
+    vals = rng.standard_normal((T, k))
+    permuted = np.empty(T * k)
+    permuted[inv.reshape(-1)] = vals.reshape(-1)
+    assert np.array_equal(permuted[inv], vals)
+    assert sorted(inv.reshape(-1)) == list(range(T * k))
+
+
+def test_permutation_empty_and_single_expert():
+    counts, offsets, perm_tok, inv = operm.permute(np.zeros((0, 2), np.int32), 4)
+    assert list(offsets) == [0, 0, 0, 0, 0] and len(perm_tok) == 0
+    counts, offsets, perm_tok, inv = operm.permute(np.zeros((5, 1), np.int32), 1)
+    assert list(perm_tok) == [0, 1, 2, 3, 4] and list(inv[:, 0]) == [0, 1, 2, 3, 4]
+
+
+def test_config_closed_forms():
+    """The K3 config printed on the pages is consistent with the page totals."""
+    import os
+    cfg = {}
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "k3_config.txt")):
+        if line.strip() and not line.startswith("#"):
+            key, val = line.split()
+            cfg[key] = val
+    E, k = int(cfg["num_experts"]), int(cfg["num_experts_per_token"])
+    I, dl = int(cfg["moe_intermediate_size"]), int(cfg["routed_expert_hidden_size"])
+    moe_layers = int(cfg["num_hidden_layers"]) - int(cfg["first_k_dense_replace"])
+    routed = moe_layers * E * 3 * dl * I
+    assert abs(routed / 1e12 - float(cfg["total_params_trillion"])) < 0.1
+    assert abs(100.0 * k / E - float(cfg["active_share_percent"])) < 0.05
+    assert int(cfg["hidden_size"]) == 2 * dl
