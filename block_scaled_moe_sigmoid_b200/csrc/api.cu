@@ -1,0 +1,496 @@
+// C ABI of the MoE layer (include/moe.h): argument checks, workspace carving, TMA
+// descriptor encoding and the launch sequence.  All arithmetic runs in the kernels of
+// kernels.cuh and gemm.cuh.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kBN = 160;      // tokens per GEMM tile (MMA N <= 160)
+constexpr int kStages = 4;    // smem pipeline depth of every GEMM
+constexpr int kPermThreads = 256;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 2-D tiled map, 128-byte swizzle.  inner = elements per row, rows = row count,
+// row_bytes = stride between rows.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+inline size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline cudaStream_t S(void* s) { return (cudaStream_t)s; }
+
+}  // namespace
+
+struct moe_plan_s {
+  int T_max, d, E, k, I, Is;
+  int num_sms = 148;
+  int last_T = 0;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  // workspace carve (byte offsets)
+  size_t o_status, o_bias0, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits,
+      o_planes, o_xq, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
+  int tokens_per_chunk() const { return kPermThreads; }
+  int nchunks(int T) const { return (T + kPermThreads - 1) / kPermThreads; }
+  template <class P>
+  P* at(size_t off) const { return (P*)(ws + off); }
+};
+
+static void carve(moe_plan_s* p) {
+  const size_t A = (size_t)p->T_max * p->k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = up(o + bytes, 1024); return r; };
+  p->o_status = take(256);
+  p->o_bias0 = take((size_t)p->E * 4);
+  p->o_chunk = take((size_t)p->nchunks(p->T_max) * p->E * 4);
+  p->o_counts = take((size_t)p->E * 4);
+  p->o_offsets = take((size_t)(p->E + 1) * 4);
+  p->o_tiles = take((size_t)(p->E + 1) * 4);
+  p->o_perm = take(A * 4);
+  p->o_inv = take(A * 4);
+  p->o_logits = take((size_t)p->T_max * p->E * 4);
+  p->o_planes = take((size_t)p->E * 3 * p->d * 2);
+  p->o_xq = take(A * p->d);
+  p->o_xs = take((size_t)(p->d / 128) * A * 4);
+  p->o_hq = take(A * p->I);
+  p->o_hs = take((size_t)(p->I / 128) * A * 4);
+  p->o_O = take(A * p->d * 2);
+  p->o_hsh = take((size_t)p->T_max * (p->Is ? p->Is : 1) * 2);
+  p->o_ys = take((size_t)p->T_max * p->d * 4);
+  p->total = o;
+}
+
+template <int KIND, int EPI>
+static cudaError_t launch_gemm(const moe_plan_s* p, const GemmArgs& a, const CUtensorMap& tA,
+                               const CUtensorMap& tB, int grid, cudaStream_t s) {
+  using Cfg = GemmCfg<KIND, kBN, kStages>;
+  auto kern = gemm_kernel<KIND, EPI, kBN, kStages>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s>>>(a, tA, tB);
+  return cudaGetLastError();
+}
+
+static GemmArgs base_args(const moe_plan_s* p) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.status = p->at<unsigned int>(p->o_status);
+  a.dense_rows = -1;
+  return a;
+}
+
+static cudaError_t set_smem_attrs() {
+  static cudaError_t st = [] {
+    cudaError_t e = cudaFuncSetAttribute(perm_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_sigmoid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    return e;
+  }();
+  return st;
+}
+
+// histogram -> scan -> placement into the plan workspace
+static cudaError_t run_permute(moe_plan_s* p, const int32_t* idx, int T, cudaStream_t s) {
+  if (set_smem_attrs() != cudaSuccess) return cudaErrorInvalidValue;
+  const int nch = p->nchunks(T);
+  int* chunk = p->at<int>(p->o_chunk);
+  perm_histogram_kernel<<<nch, 256, p->E * 4, s>>>(idx, T, p->k, p->E, p->tokens_per_chunk(), chunk,
+                                                   p->at<unsigned int>(p->o_status));
+  perm_scan_kernel<<<1, 1024, (2 * p->E + 32) * 4, s>>>(chunk, nch, p->E, kBN, p->at<int>(p->o_counts),
+                                                         p->at<int>(p->o_offsets), p->at<int>(p->o_tiles));
+  perm_place_kernel<<<nch, kPermThreads, (kPermThreads / 32) * p->E * 4, s>>>(
+      idx, T, p->k, p->E, p->tokens_per_chunk(), chunk, p->at<int>(p->o_perm), p->at<int>(p->o_inv));
+  return cudaGetLastError();
+}
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_ALIGNMENT: return "misaligned pointer";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_NOT_INITIALIZED: return "no workspace attached";
+    case MOE_ERR_DEVICE_FAULT: return "device flagged invalid input";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared, moe_act_t act,
+                             moe_bias_mode_t bias_mode, int flags, moe_plan_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (act != MOE_ACT_SILU_GLU || bias_mode != MOE_BIAS_LOGIT || flags != 0) return MOE_ERR_INVALID_ARG;
+  if (T_max < 0 || d <= 0 || E <= 0 || k <= 0 || I <= 0 || I_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (d % 128 || I % 128 || I_shared % 128 || k > E || k > 32 || E > 4096)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T_max * k > (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  moe_plan_s* p = new moe_plan_s();
+  p->T_max = T_max; p->d = d; p->E = E; p->k = k; p->I = I; p->Is = I_shared;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+      p->num_sms = sms;
+  }
+  carve(p);
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_workspace_bytes(moe_plan_t p, size_t* bytes) {
+  if (!p || !bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = p->total;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_set_workspace(moe_plan_t p, void* dev_ptr, size_t bytes) {
+  if (!p || !dev_ptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(dev_ptr, 256)) return MOE_ERR_ALIGNMENT;
+  if (bytes < p->total) return MOE_ERR_INVALID_ARG;
+  p->ws = (char*)dev_ptr;
+  p->ws_bytes = bytes;
+  if (cudaMemset(p->ws + p->o_status, 0, 256) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_check(moe_plan_t p, void* stream, unsigned int* bits) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  unsigned int v = 0;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, p->ws + p->o_status, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(p->ws + p->o_status, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (bits) *bits = v;
+  if (v & MOE_DEV_ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (v) return MOE_ERR_DEVICE_FAULT;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_destroy(moe_plan_t p) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  delete p;
+  return MOE_OK;
+}
+
+moe_status_t moe_quant_mxfp8(const void* x, int rows, int cols, uint8_t* q, uint8_t* sc, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 32) return rows < 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !sc) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16)) return MOE_ERR_ALIGNMENT;
+  const long long n = (long long)rows * (cols / 32);
+  const int threads = 256;
+  quant_mxfp8_kernel<<<(unsigned)((n + threads - 1) / threads), threads, 0, S(stream)>>>(
+      (const uint16_t*)x, rows, cols, q, sc);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_permute(moe_plan_t p, const int32_t* idx, int T, int32_t* counts, int32_t* offsets,
+                         int32_t* perm_tok, int32_t* inv, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > p->T_max) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !offsets || (T > 0 && (!idx || !perm_tok || !inv))) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = S(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, p->E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(offsets, 0, (p->E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (run_permute(p, idx, T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t A = (size_t)T * p->k;
+  if (cudaMemcpyAsync(counts, p->ws + p->o_counts, p->E * 4, cudaMemcpyDeviceToDevice, s) ||
+      cudaMemcpyAsync(offsets, p->ws + p->o_offsets, (p->E + 1) * 4, cudaMemcpyDeviceToDevice, s) ||
+      cudaMemcpyAsync(perm_tok, p->ws + p->o_perm, A * 4, cudaMemcpyDeviceToDevice, s) ||
+      cudaMemcpyAsync(inv, p->ws + p->o_inv, A * 4, cudaMemcpyDeviceToDevice, s))
+    return MOE_ERR_CUDA;
+  p->last_T = T;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, const float* bias,
+                       int32_t* idx, float* w, float* logits_opt, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > p->T_max) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !W_r || !idx || !w) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(W_r, 16)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t s = S(stream);
+  const int d = p->d, E = p->E;
+  __nv_bfloat16* planes = p->at<__nv_bfloat16>(p->o_planes);
+  float* z = logits_opt ? logits_opt : p->at<float>(p->o_logits);
+  if (!aligned(z, 16)) return MOE_ERR_ALIGNMENT;
+  router_split_kernel<<<dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s>>>(W_r, d, E, planes);
+  float* zero_bias = nullptr;
+  if (!bias) {
+    zero_bias = p->at<float>(p->o_bias0);
+    if (cudaMemsetAsync(zero_bias, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  CUtensorMap tA, tB;
+  if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, planes, 3ull * d, E, 3ull * d * 2, 64, 256) ||
+      !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64, 32))
+    return MOE_ERR_CUDA;
+  GemmArgs a = base_args(p);
+  a.dense_rows = T;
+  a.num_groups = 1;
+  a.M_total = E;
+  a.m_tiles = (E + 255) / 256;
+  a.k_tiles = 3 * d / 64;
+  a.kb_wrap = d / 64;
+  a.B_rows = T;
+  a.out0 = z;
+  a.ld_out = E;
+  a.bias = bias ? bias : zero_bias;
+  const int tiles = ((T + kBN - 1) / kBN) * a.m_tiles;
+  if (launch_gemm<KIND_BF16, EPI_LOGITS>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (set_smem_attrs() != cudaSuccess) return MOE_ERR_CUDA;
+  const int wpb = 8;
+  topk_sigmoid_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * E * 4, s>>>(z, T, E, p->k, idx, w);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  p->last_T = T;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx, const float* w,
+                         const moe_experts_mxfp4* ex, const moe_shared_bf16* sh, void* y, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > p->T_max) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return MOE_OK;
+  if (!x || !idx || !w || !ex || !y || !ex->w_gu || !ex->s_gu || !ex->w_dn || !ex->s_dn)
+    return MOE_ERR_INVALID_ARG;
+  if ((p->Is > 0) != (sh != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (sh && (!sh->w_gu || !sh->w_dn)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ex->w_gu, 256) || !aligned(ex->w_dn, 256) ||
+      !aligned(ex->s_gu, 16) || !aligned(ex->s_dn, 16) ||
+      (sh && (!aligned(sh->w_gu, 16) || !aligned(sh->w_dn, 16))))
+    return MOE_ERR_ALIGNMENT;
+  cudaStream_t s = S(stream);
+  const int d = p->d, E = p->E, k = p->k, I = p->I, Is = p->Is;
+  const int A = T * k;
+
+  // a4: group assignments by expert
+  if (run_permute(p, idx, T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // a1: quantise x to MXFP8 and scatter rows into expert order
+  uint8_t* xq = p->at<uint8_t>(p->o_xq);
+  uint32_t* xs = p->at<uint32_t>(p->o_xs);
+  {
+    const long long n = (long long)T * (d / 32);
+    quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        (const uint16_t*)x, T, d, k, p->at<int>(p->o_inv), A, xq, xs);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  uint8_t* hq = p->at<uint8_t>(p->o_hq);
+  uint32_t* hs = p->at<uint32_t>(p->o_hs);
+  __nv_bfloat16* O = p->at<__nv_bfloat16>(p->o_O);
+  // a5/a6: gate/up grouped GEMM, SiLU-GLU and MXFP8 requantisation in the epilogue
+  {
+    CUtensorMap tA, tB;
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, d, (uint64_t)E * 2 * I, d / 2, 128, 256) ||
+        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, d, A, d, 128, 32))
+      return MOE_ERR_CUDA;
+    GemmArgs a = base_args(p);
+    a.counts = p->at<int>(p->o_counts);
+    a.offsets = p->at<int>(p->o_offsets);
+    a.tile_prefix = p->at<int>(p->o_tiles);
+    a.num_groups = E;
+    a.M_total = 2 * I;
+    a.m_tiles = 2 * I / 256;
+    a.k_tiles = d / 128;
+    a.kb_wrap = a.k_tiles;
+    a.B_rows = A;
+    a.sfa = (const uint8_t*)ex->s_gu;
+    a.sfb = xs;
+    a.out0 = hq;
+    a.out1 = hs;
+    a.ld_out = I;
+    if (launch_gemm<KIND_MX, EPI_GLU_MX8>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // a7: down grouped GEMM -> O (bf16, expert order)
+  {
+    CUtensorMap tA, tB;
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_dn, I, (uint64_t)E * d, I / 2, 128, 256) ||
+        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, A, I, 128, 32))
+      return MOE_ERR_CUDA;
+    GemmArgs a = base_args(p);
+    a.counts = p->at<int>(p->o_counts);
+    a.offsets = p->at<int>(p->o_offsets);
+    a.tile_prefix = p->at<int>(p->o_tiles);
+    a.num_groups = E;
+    a.M_total = d;
+    a.m_tiles = (d + 255) / 256;
+    a.k_tiles = I / 128;
+    a.kb_wrap = a.k_tiles;
+    a.B_rows = A;
+    a.sfa = (const uint8_t*)ex->s_dn;
+    a.sfb = hs;
+    a.out0 = O;
+    a.ld_out = d;
+    if (launch_gemm<KIND_MX, EPI_BF16>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // a8: shared expert (bf16)
+  float* ys = nullptr;
+  if (sh) {
+    __nv_bfloat16* hsh = p->at<__nv_bfloat16>(p->o_hsh);
+    ys = p->at<float>(p->o_ys);
+    CUtensorMap tA, tB;
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sh->w_gu, d, 2ull * Is, (uint64_t)d * 2, 64, 256) ||
+        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64, 32))
+      return MOE_ERR_CUDA;
+    GemmArgs a = base_args(p);
+    a.dense_rows = T;
+    a.num_groups = 1;
+    a.M_total = 2 * Is;
+    a.m_tiles = 2 * Is / 256;
+    a.k_tiles = d / 64;
+    a.kb_wrap = a.k_tiles;
+    a.B_rows = T;
+    a.out0 = hsh;
+    a.ld_out = Is;
+    int tiles = ((T + kBN - 1) / kBN) * a.m_tiles;
+    if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    CUtensorMap tA2, tB2;
+    if (!make_map(&tA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sh->w_dn, Is, d, (uint64_t)Is * 2, 64, 256) ||
+        !make_map(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hsh, Is, T, (uint64_t)Is * 2, 64, 32))
+      return MOE_ERR_CUDA;
+    GemmArgs b = base_args(p);
+    b.dense_rows = T;
+    b.num_groups = 1;
+    b.M_total = d;
+    b.m_tiles = (d + 255) / 256;
+    b.k_tiles = Is / 64;
+    b.kb_wrap = b.k_tiles;
+    b.B_rows = T;
+    b.out0 = ys;
+    b.ld_out = d;
+    tiles = ((T + kBN - 1) / kBN) * b.m_tiles;
+    if (launch_gemm<KIND_BF16, EPI_F32>(p, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  // a9: weighted combine with the shared output
+  combine_kernel<<<T, 128, k * 8, s>>>(O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  p->last_T = T;
+  return MOE_OK;
+}
+
+moe_status_t moe_expert_bytes(int d, int I, int E, size_t* w_gu, size_t* s_gu, size_t* w_dn, size_t* s_dn) {
+  if (d <= 0 || I <= 0 || E <= 0 || !w_gu || !s_gu || !w_dn || !s_dn) return MOE_ERR_INVALID_ARG;
+  if (d % 128 || I % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  *w_gu = (size_t)E * 2 * I * (d / 2);
+  *s_gu = (size_t)E * (2 * I / 256) * (d / 128) * 1024;
+  *w_dn = (size_t)E * d * (I / 2);
+  *s_dn = (size_t)E * ((d + 255) / 256) * (I / 128) * 1024;
+  return MOE_OK;
+}
+
+moe_status_t moe_pack_expert_mxfp4(int d, int I, int e, const float* wg, const float* wu, const float* wd,
+                                   const moe_experts_mxfp4* dst, void* stream) {
+  if (d <= 0 || I <= 0 || e < 0 || !wg || !wu || !wd || !dst || !dst->w_gu || !dst->s_gu || !dst->w_dn ||
+      !dst->s_dn)
+    return MOE_ERR_INVALID_ARG;
+  if (d % 128 || I % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(wg, 16) || !aligned(wu, 16) || !aligned(wd, 16)) return MOE_ERR_ALIGNMENT;
+  cudaStream_t s = S(stream);
+  const size_t gu_w = (size_t)2 * I * (d / 2), gu_s = (size_t)(2 * I / 256) * (d / 128) * 1024;
+  const size_t dn_w = (size_t)d * (I / 2), dn_s = (size_t)((d + 255) / 256) * (I / 128) * 1024;
+  uint8_t* wgu = (uint8_t*)dst->w_gu + (size_t)e * gu_w;
+  uint8_t* sgu = (uint8_t*)dst->s_gu + (size_t)e * gu_s;
+  uint8_t* wdn = (uint8_t*)dst->w_dn + (size_t)e * dn_w;
+  uint8_t* sdn = (uint8_t*)dst->s_dn + (size_t)e * dn_s;
+  // the down scales' last tile may have an unused half: keep it defined
+  if (cudaMemsetAsync(sdn, 0, dn_s, s) != cudaSuccess) return MOE_ERR_CUDA;
+  long long n = 2ll * I * (d / 32);
+  pack_mxfp4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(wg, wu, I, d, 1, wgu, sgu);
+  n = (long long)d * (I / 32);
+  pack_mxfp4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(wd, nullptr, d, I, 0, wdn, sdn);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_pack_shared_bf16(int d, int Is, const void* wg, const void* wu, const void* wd,
+                                  const moe_shared_bf16* dst, void* stream) {
+  if (d <= 0 || Is <= 0 || !wg || !wu || !wd || !dst || !dst->w_gu || !dst->w_dn) return MOE_ERR_INVALID_ARG;
+  if (d % 128 || Is % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = S(stream);
+  const size_t row = (size_t)d * 2;
+  for (int b = 0; b < Is / 128; ++b) {
+    char* out = (char*)dst->w_gu + (size_t)256 * b * row;
+    if (cudaMemcpyAsync(out, (const char*)wg + (size_t)128 * b * row, 128 * row, cudaMemcpyDeviceToDevice, s) ||
+        cudaMemcpyAsync(out + 128 * row, (const char*)wu + (size_t)128 * b * row, 128 * row,
+                        cudaMemcpyDeviceToDevice, s))
+      return MOE_ERR_CUDA;
+  }
+  if (cudaMemcpyAsync(dst->w_dn, wd, (size_t)d * Is * 2, cudaMemcpyDeviceToDevice, s)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes) {
+  if (!p || !ptr || !bytes) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  const size_t A = (size_t)p->last_T * p->k, T = p->last_T;
+  size_t off, n;
+  switch (which) {
+    case 0: off = p->o_xq; n = A * p->d; break;
+    case 1: off = p->o_xs; n = (p->d / 128) * A * 4; break;
+    case 2: off = p->o_hq; n = A * p->I; break;
+    case 3: off = p->o_hs; n = (p->I / 128) * A * 4; break;
+    case 4: off = p->o_O; n = A * p->d * 2; break;
+    case 5: off = p->o_ys; n = T * p->d * 4; break;
+    case 6: off = p->o_logits; n = T * p->E * 4; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  *ptr = p->ws + off;
+  *bytes = n;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,375 @@
+// Persistent, warp-specialised grouped GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// Computes, per tile, D = A_tile * B_tile^T where
+//   A = weight rows (output channels, K-major), 256 rows per tile as two 128-row halves
+//   B = token rows (K-major), up to BN_MAX rows per tile (the MMA's N dimension)
+// so the accumulator's TMEM lane is the output channel and its column is the token
+// ("swap-AB": a Kimi-K3 expert sees ~146 tokens at T=8192, which fits one N tile
+// while the weights fill the 128-row M dimension).
+//
+// Kinds:
+//   KIND_MX:   tcgen05.mma kind::mxf8f6f4.block_scale, A = E2M1 (MXFP4 weights, loaded by
+//              TMA with the 16U4_ALIGN16B unpacking type), B = E4M3 (MXFP8 activations),
+//              one E8M0 scale per 32 K-elements on both sides, fp32 accumulation.
+//   KIND_BF16: tcgen05.mma kind::f16 with bf16 A and B, fp32 accumulation.
+//
+// Groups: rows of B are grouped (one group per expert, contiguous rows
+// [offsets[g], offsets[g+1])); each group is split into ceil(rows / BN_MAX) tiles of
+// balanced size.  "dense" mode is one implicit group of dense_rows rows.  Tile t
+// covers group-tile t / m_tiles and weight m-tile t % m_tiles, so CTAs running at the
+// same time share the group's B rows through L2.
+//
+// Roles (320 threads): warp 0 loads (TMA for A/B tiles, bulk copy for A scales,
+// cp.async for B scales), warp 1 owns TMEM and one lane issues the MMAs, warps 2..9
+// run the epilogue (lane quarter = warp % 4).
+#pragma once
+#include "ptx.cuh"
+
+namespace moe {
+
+enum { KIND_MX = 0, KIND_BF16 = 1 };
+enum {
+  EPI_GLU_MX8 = 0,   // a = silu(gate) * up, requantised to MXFP8 along the channels
+  EPI_GLU_BF16 = 1,  // a = silu(gate) * up, stored as bf16
+  EPI_BF16 = 2,      // D stored as bf16
+  EPI_F32 = 3,       // D stored as fp32
+  EPI_LOGITS = 4     // D + bias[channel] stored as fp32
+};
+
+struct GemmArgs {
+  const int* counts;       // [G] rows per group (routed mode)
+  const int* offsets;      // [G+1] first row of each group
+  const int* tile_prefix;  // [G+1] first group-tile of each group
+  int num_groups;
+  int dense_rows;   // >= 0: one implicit group with this many rows (no group arrays)
+  int M_total;      // A rows per group (output channels)
+  int m_tiles;      // ceil(M_total / 256)
+  int k_tiles;      // K / BK
+  int kb_wrap;      // B's K-tile coordinate is taken modulo kb_wrap
+  int B_rows;       // rows of the B tensor
+  const uint8_t* sfa;   // KIND_MX: A scales, [G][m_tiles][k_tiles][2 halves][512 B atom]
+  const uint32_t* sfb;  // KIND_MX: B scales, words [k_tiles][B_rows], byte j = K-block 4kt+j
+  void* out0;
+  void* out1;
+  int ld_out;           // elements per output row
+  const float* bias;    // EPI_LOGITS
+  unsigned int* status;
+};
+
+template <int KIND, int BN_MAX, int STAGES>
+struct GemmCfg {
+  static constexpr int BM = 256;                               // two 128-row halves
+  static constexpr int BK = KIND == KIND_MX ? 128 : 64;        // elements per K tile (128 B rows)
+  static constexpr int A_BYTES = BM * 128;                     // smem (FP4 padded to 1 B/elem)
+  static constexpr int B_BYTES = BN_MAX * 128;
+  static constexpr int SFA_BYTES = KIND == KIND_MX ? 1024 : 0;
+  static constexpr int SFB_ATOMS = (BN_MAX + 127) / 128;
+  static constexpr int SFB_BYTES = KIND == KIND_MX ? SFB_ATOMS * 512 : 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int A_TX = KIND == KIND_MX ? BM * BK / 2 : BM * BK * 2;  // global bytes
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+  static constexpr int TMEM_SFA = 2 * BN_MAX;                  // 4 columns per half
+  static constexpr int TMEM_SFB = 2 * BN_MAX + 8;              // 4 columns per 128 B rows
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int NUM_THREADS = 320;
+  static_assert(BN_MAX % 32 == 0 && BN_MAX <= 256, "BN_MAX");
+  static_assert(TMEM_SFB + 4 * SFB_ATOMS <= TMEM_COLS, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct TileInfo {
+  int grp, mt, row0, n_valid, n_mma;
+};
+
+__device__ __forceinline__ int gemm_num_tiles(const GemmArgs& a, int bn_max) {
+  if (a.dense_rows >= 0) return ((a.dense_rows + bn_max - 1) / bn_max) * a.m_tiles;
+  return __ldg(a.tile_prefix + a.num_groups) * a.m_tiles;
+}
+
+__device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, int t, TileInfo& ti) {
+  const int gt = t / a.m_tiles;
+  ti.mt = t - gt * a.m_tiles;
+  int grp, nt, ntiles, Me, base;
+  if (a.dense_rows >= 0) {
+    grp = 0;
+    nt = gt;
+    Me = a.dense_rows;
+    ntiles = (Me + bn_max - 1) / bn_max;
+    base = 0;
+  } else {
+    int lo = 0, hi = a.num_groups - 1;  // last group whose first tile is <= gt
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(a.tile_prefix + mid) <= gt) lo = mid; else hi = mid - 1;
+    }
+    grp = lo;
+    const int tp = __ldg(a.tile_prefix + grp);
+    nt = gt - tp;
+    ntiles = __ldg(a.tile_prefix + grp + 1) - tp;
+    Me = __ldg(a.counts + grp);
+    base = __ldg(a.offsets + grp);
+  }
+  int n_per = (Me + ntiles - 1) / ntiles;
+  n_per = (n_per + 15) & ~15;
+  ti.grp = grp;
+  ti.row0 = base + nt * n_per;
+  ti.n_valid = min(n_per, Me - nt * n_per);
+  ti.n_mma = (ti.n_valid + 15) & ~15;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+
+// MXFP8 (E4M3) encoding of v with block scale exponent from the block's amax bits.
+__device__ __forceinline__ int mx_exp_e4m3(uint32_t amax_bits) {
+  const int ex = (int)((amax_bits >> 23) & 0xFF);
+  const int e = (ex == 0) ? -127 : ex - 127 - 8;   // floor(log2 amax) - emax(E4M3)
+  return max(e, -127);
+}
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int KIND, int EPI, int BN_MAX, int STAGES>
+__global__ void __launch_bounds__(320, 1)
+    gemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA,
+                const __grid_constant__ CUtensorMap tmB) {
+  using C = GemmCfg<KIND, BN_MAX, STAGES>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ctrl = smem + STAGES * C::STAGE_BYTES;
+  uint64_t* full_bar = (uint64_t*)ctrl;
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* acc_full = empty_bar + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain_bar = acc_empty + 1;
+  uint32_t* tmem_holder = (uint32_t*)(drain_bar + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 33 : 1);
+      mbar_init(smem_u32(empty_bar + s), 1);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_empty), 8);
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int num_tiles = gemm_num_tiles(args, BN_MAX);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    const uint64_t pol_a = policy_evict_first();  // weights stream through once
+    const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      TileInfo ti;
+      gemm_decode_tile(args, BN_MAX, t, ti);
+      const int a_row = ti.grp * args.M_total + ti.mt * C::BM;
+      const int nB = (ti.n_mma + 31) >> 5;
+      bool ok = true;
+      for (int kt = 0; kt < args.k_tiles; ++kt) {
+        if (lane == 0) ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        uint8_t* sA = smem + stage * C::STAGE_BYTES;
+        uint8_t* sB = sA + C::A_BYTES;
+        uint8_t* sSFA = sB + C::B_BYTES;
+        uint8_t* sSFB = sSFA + C::SFA_BYTES;
+        const uint32_t fb = smem_u32(full_bar + stage);
+        if constexpr (KIND == KIND_MX) {
+          // B scales: one 32-bit word (4 K-blocks) per token row, into the MMA's
+          // scale-factor atom layout: row n -> atom n/128, byte (n%32)*16 + ((n%128)/32)*4.
+          const uint32_t* src = args.sfb + (size_t)kt * args.B_rows + ti.row0;
+          for (int n = lane; n < ti.n_valid; n += 32) {
+            const uint32_t off = (n >> 7) * 512 + (n & 31) * 16 + ((n & 127) >> 5) * 4;
+            cp_async_4(smem_u32(sSFB + off), src + n);
+          }
+          cp_async_mbar_arrive_noinc(fb);
+        }
+        if (lane == 0) {
+          const uint32_t tx = C::A_TX + nB * 4096 + C::SFA_BYTES;
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
+          if constexpr (KIND == KIND_MX) {
+            const uint8_t* sfa_src =
+                args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::
+                    "r"(smem_u32(sSFA)),
+                "l"(sfa_src), "r"(fb)
+                : "memory");
+          }
+          const int kb = kt % args.kb_wrap;
+          for (int i = 0; i < nB; ++i)
+            tma_load_2d(smem_u32(sB + i * 4096), &tmB, fb, kb * C::BK, ti.row0 + 32 * i, pol_b);
+        }
+        __syncwarp();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        TileInfo ti;
+        gemm_decode_tile(args, BN_MAX, t, ti);
+        const bool h1 = ti.mt * C::BM + 128 < args.M_total;
+        ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          if constexpr (KIND == KIND_MX) {
+            const uint32_t sSFA = sB + C::B_BYTES;
+            const uint32_t sSFB = sSFA + C::SFA_BYTES;
+            tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFA, smem_desc(sSFA, 16, 128, 0));
+            if (h1) tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFA + 4, smem_desc(sSFA + 512, 16, 128, 0));
+            const int atoms = (ti.n_mma + 127) >> 7;
+            for (int a = 0; a < atoms; ++a)
+              tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFB + 4 * a, smem_desc(sSFB + 512 * a, 16, 128, 0));
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t bdesc = smem_desc(sB + 32 * j, 16, 1024, 2);
+            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              if (h == 1 && !h1) continue;
+              const uint64_t adesc = smem_desc(sA + h * 16384 + 32 * j, 16, 1024, 2);
+              const uint32_t d_tmem = tmem_base + h * BN_MAX;
+              if constexpr (KIND == KIND_MX) {
+                const uint32_t idesc = idesc_mx_e2m1_e4m3(128, ti.n_mma, j, j);
+                const uint32_t sfa = (tmem_base + C::TMEM_SFA + 4 * h) | ((uint32_t)j << 30);
+                const uint32_t sfb = (tmem_base + C::TMEM_SFB) | ((uint32_t)j << 30);
+                mma_mxf8f6f4(d_tmem, adesc, bdesc, idesc, sfa, sfb, acc);
+              } else {
+                mma_bf16(d_tmem, adesc, bdesc, idesc_bf16(128, ti.n_mma), acc);
+              }
+            }
+          }
+          tc_commit(smem_u32(empty_bar + stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(acc_full));
+        acc_phase ^= 1;
+      }
+      // make sure every MMA this thread issued has finished before TMEM is released
+      tc_commit(smem_u32(drain_bar));
+      mbar_wait(smem_u32(drain_bar), 0, args.status, abort_flag);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int sub = (warp - 2) >> 2;   // 0 or 1
+    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      TileInfo ti;
+      gemm_decode_tile(args, BN_MAX, t, ti);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(smem_u32(acc_full), acc_phase, args.status, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const int nchunks = ti.n_mma >> 4;
+      if constexpr (EPI == EPI_GLU_MX8 || EPI == EPI_GLU_BF16) {
+        const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
+        for (int c = sub; c < nchunks; c += 2) {
+          uint32_t g[16], u[16];
+          tmem_ld16(lane_base + c * 16, g);
+          tmem_ld16(lane_base + BN_MAX + c * 16, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = c * 16 + i;
+            if (n >= ti.n_valid) break;
+            const float gv = __uint_as_float(g[i]);
+            const float a = silu_f(gv) * __uint_as_float(u[i]);
+            const size_t row = (size_t)(ti.row0 + n);
+            if constexpr (EPI == EPI_GLU_MX8) {
+              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a) & 0x7FFFFFFFu);
+              const int e = mx_exp_e4m3(amax);
+              const float qv = a * __uint_as_float((uint32_t)(127 - e) << 23);
+              const uint32_t code = f32x2_to_e4m3x2(qv, 0.0f) & 0xFFu;
+              ((uint8_t*)args.out0)[row * args.ld_out + ch] = (uint8_t)code;
+              if (lane == 0)
+                ((uint8_t*)args.out1)[((size_t)ti.mt * args.B_rows + row) * 4 + q] = (uint8_t)(e + 127);
+            } else {
+              ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a);
+            }
+          }
+        }
+      } else {
+        const int h = sub;
+        const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
+        const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
+        if (half_ok) {
+          const bool ch_ok = ch < args.M_total;
+          float bias = 0.0f;
+          if constexpr (EPI == EPI_LOGITS) bias = ch_ok ? __ldg(args.bias + ch) : 0.0f;
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[16];
+            tmem_ld16(lane_base + h * BN_MAX + c * 16, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int n = c * 16 + i;
+              if (n >= ti.n_valid) break;
+              if (!ch_ok) continue;
+              const size_t o = (size_t)(ti.row0 + n) * args.ld_out + ch;
+              const float x = __uint_as_float(v[i]);
+              if constexpr (EPI == EPI_BF16) ((__nv_bfloat16*)args.out0)[o] = __float2bfloat16_rn(x);
+              else ((float*)args.out0)[o] = x + bias;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+      acc_phase ^= 1;
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // let any bulk copies still in flight land before the CTA's shared memory goes away
+    __nanosleep(100000);
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,411 @@
+// CUDA-core kernels of the MoE layer: MXFP8 quantiser (plain and scatter-to-expert-order),
+// token->expert histogram / scan / stable placement, sigmoid top-k selection,
+// weighted combine, and the setup-time weight packers (MXFP4 experts, bf16 router planes).
+#pragma once
+#include "ptx.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- MX element conversion
+// OCP MX block rule: scale exponent e = floor(log2(amax)) - emax, clamped below at -127;
+// elements are round-to-nearest-even, saturating, sign kept (-0 stays -0).
+__device__ __forceinline__ int mx_scale_exp(float amax, int emax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ex = (int)((b >> 23) & 0xFF);
+  const int e = (ex == 0) ? -127 : ex - 127 - emax;  // subnormal or zero amax -> clamp
+  return max(e, -127);
+}
+__device__ __forceinline__ float pow2_neg(int e) {  // 2^-e for e in [-127, 126]
+  return __uint_as_float((uint32_t)(127 - e) << 23);
+}
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}\n"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One 32-element bf16 block -> 32 E4M3 bytes (as 8 words) + scale byte.
+__device__ __forceinline__ uint32_t quant_block_e4m3(const uint4 (&in)[4], uint32_t (&out)[8]) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {in[i].x, in[i].y, in[i].z, in[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[i * 8 + 2 * j] = __uint_as_float(w[j] << 16);
+      v[i * 8 + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = mx_scale_exp(amax, 8);
+  const float s = pow2_neg(e);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = cvt_e4m3x2(v[4 * i] * s, v[4 * i + 1] * s);
+    const uint32_t hi = cvt_e4m3x2(v[4 * i + 2] * s, v[4 * i + 3] * s);
+    out[i] = lo | (hi << 16);
+  }
+  return (uint32_t)(e + 127);
+}
+
+// x bf16 [rows][cols] -> q E4M3 [rows][cols], scale E8M0 [rows][cols/32].
+__global__ void quant_mxfp8_kernel(const uint16_t* __restrict__ x, int rows, int cols,
+                                   uint8_t* __restrict__ q, uint8_t* __restrict__ sc) {
+  const int nb = cols >> 5;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)rows * nb) return;
+  const long long r = gid / nb;
+  const int b = (int)(gid - r * nb);
+  const uint4* src = (const uint4*)(x + r * cols + b * 32);
+  uint4 in[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
+  uint32_t out[8];
+  const uint32_t s = quant_block_e4m3(in, out);
+  uint4* dst = (uint4*)(q + r * cols + b * 32);
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  sc[r * nb + b] = (uint8_t)s;
+}
+
+// Quantise token rows and write each to its k positions in expert order:
+// xq[inv[t][j]][:] and the scale words xs[(block/4)][inv[t][j]] (byte block%4).
+// Requires cols % 128 == 0 so four consecutive threads share a row and one word.
+__global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int cols, int k,
+                                     const int* __restrict__ inv, int A_rows,
+                                     uint8_t* __restrict__ xq, uint32_t* __restrict__ xs) {
+  const int nb = cols >> 5;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool active = gid < (long long)T * nb;
+  const long long t = active ? gid / nb : 0;
+  const int b = active ? (int)(gid - t * nb) : 0;
+  uint4 in[4] = {};
+  if (active) {
+    const uint4* src = (const uint4*)(x + t * cols + b * 32);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
+  }
+  uint32_t out[8];
+  const uint32_t s = quant_block_e4m3(in, out);
+  // gather the 4 scale bytes of blocks 4m..4m+3 into lane 4m's word
+  const int l = threadIdx.x & 31;
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
+  if (!active) return;
+  const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  const uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
+  const uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
+  for (int j = 0; j < k; ++j) {
+    const int p = __ldg(inv + t * k + j);
+    if (p < 0 || p >= A_rows) continue;
+    uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
+    dst[0] = o0;
+    dst[1] = o1;
+    if ((l & 3) == 0) xs[(size_t)(b >> 2) * A_rows + p] = word;
+  }
+}
+
+// ---------------------------------------------------------------- permutation
+// Chunks of TPC tokens (32 per warp); chunk_counts[c][e] = assignments of chunk c to e.
+__global__ void perm_histogram_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                      int tokens_per_chunk, int* __restrict__ chunk_counts,
+                                      unsigned int* status) {
+  extern __shared__ int cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * tokens_per_chunk;
+  const int n = min(tokens_per_chunk, T - t0) * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = __ldg(idx + (size_t)t0 * k + i);
+    if (e < 0 || e >= E) {
+      atomicOr(status, MOE_DEV_ERR_BOUNDS);
+      continue;
+    }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Block-wide exclusive scan of n <= 4 * blockDim.x values in place (1024 threads).
+__device__ void block_exclusive_scan(int* vals, int n, int* warp_tot) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int i0 = threadIdx.x * per;
+  int local = 0;
+  for (int i = 0; i < per; ++i)
+    if (i0 + i < n) local += vals[i0 + i];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    warp_tot[lane] = inc - v;
+  }
+  __syncthreads();
+  int run = warp_tot[w] + incl - local;
+  for (int i = 0; i < per; ++i)
+    if (i0 + i < n) {
+      const int v = vals[i0 + i];
+      vals[i0 + i] = run;
+      run += v;
+    }
+  __syncthreads();
+}
+
+// Single CTA: counts, offsets (exclusive scan), per-chunk bases, and the GEMM tile prefix
+// (ceil(count / bn_max) tiles per expert).
+__global__ void perm_scan_kernel(int* __restrict__ chunk_counts, int nchunks, int E, int bn_max,
+                                 int* __restrict__ counts, int* __restrict__ offsets,
+                                 int* __restrict__ tile_prefix) {
+  extern __shared__ int sh[];
+  int* s_off = sh;            // E
+  int* s_tiles = sh + E;      // E
+  int* warp_tot = sh + 2 * E; // 32
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      int* p = chunk_counts + (size_t)c * E + e;
+      const int v = *p;
+      *p = run;
+      run += v;
+    }
+    counts[e] = run;
+    s_off[e] = run;
+    s_tiles[e] = (run + bn_max - 1) / bn_max;
+  }
+  __syncthreads();
+  const int total_rows_last = s_off[E - 1];
+  const int total_tiles_last = s_tiles[E - 1];
+  __syncthreads();
+  block_exclusive_scan(s_off, E, warp_tot);
+  block_exclusive_scan(s_tiles, E, warp_tot);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    offsets[e] = s_off[e];
+    tile_prefix[e] = s_tiles[e];
+    for (int c = 0; c < nchunks; ++c) chunk_counts[(size_t)c * E + e] += s_off[e];
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = s_off[E - 1] + total_rows_last;
+    tile_prefix[E] = s_tiles[E - 1] + total_tiles_last;
+  }
+}
+
+// Stable placement: position of (t, j) = base of (chunk, expert) + number of earlier
+// tokens of the chunk that also chose that expert.  Warp w of a chunk owns tokens
+// 32w..32w+31 and builds a per-expert lane mask; ranks come from popcounts.
+__global__ void perm_place_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                  int tokens_per_chunk, const int* __restrict__ chunk_base,
+                                  int* __restrict__ perm_tok, int* __restrict__ inv) {
+  extern __shared__ uint32_t masks[];  // [warps][E]
+  const int warps = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < warps * E; i += blockDim.x) masks[i] = 0;
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * tokens_per_chunk + threadIdx.x;
+  const bool valid = threadIdx.x < tokens_per_chunk && t < T;
+  if (valid)
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(idx + (size_t)t * k + j);
+      if (e >= 0 && e < E) atomicOr(&masks[w * E + e], 1u << lane);
+    }
+  __syncthreads();
+  if (!valid) return;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int* base = chunk_base + (size_t)blockIdx.x * E;
+  for (int j = 0; j < k; ++j) {
+    const int e = __ldg(idx + (size_t)t * k + j);
+    if (e < 0 || e >= E) {
+      inv[(size_t)t * k + j] = -1;
+      continue;
+    }
+    int r = __popc(masks[w * E + e] & lt);
+    for (int w2 = 0; w2 < w; ++w2) r += __popc(masks[w2 * E + e]);
+    const int p = base[e] + r;
+    inv[(size_t)t * k + j] = p;
+    perm_tok[p] = t;
+  }
+}
+
+// ---------------------------------------------------------------- top-k
+// One warp per token: k rounds of a warp arg-max over the logits (descending value,
+// lower index on ties), then sigmoid weights renormalised to sum 1.
+__global__ void topk_sigmoid_kernel(const float* __restrict__ z, int T, int E, int k,
+                                    int* __restrict__ idx_out, float* __restrict__ w_out) {
+  extern __shared__ float zs[];  // [warps][E]
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + w;
+  if (t >= T) return;
+  float* row = zs + (size_t)w * E;
+  for (int e = lane; e < E; e += 32) row[e] = __ldg(z + (size_t)t * E + e);
+  __syncwarp();
+  float ssum = 0.0f, my_s = 0.0f;
+  int my_i = -1;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      const float v = row[e];
+      if (v > bv) { bv = v; bi = e; }  // ascending e: first max kept on ties
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    const float s = 1.0f / (1.0f + expf(-bv));
+    ssum += s;
+    if (lane == r) { my_s = s; my_i = bi; }
+    if (lane == 0) row[bi] = -INFINITY;
+    __syncwarp();
+  }
+  if (lane < k) {
+    idx_out[(size_t)t * k + lane] = my_i;
+    w_out[(size_t)t * k + lane] = my_s / ssum;
+  }
+}
+
+// ---------------------------------------------------------------- combine
+// y[t] = bf16( y_shared[t] + sum_j w[t][j] * O[inv[t][j]] ), fp32 sums in slot order.
+__global__ void combine_kernel(const __nv_bfloat16* __restrict__ O, const float* __restrict__ ys,
+                               const float* __restrict__ w, const int* __restrict__ inv, int T,
+                               int d, int k, __nv_bfloat16* __restrict__ y) {
+  const int t = blockIdx.x;
+  extern __shared__ int s_inv[];
+  float* s_w = (float*)(s_inv + k);
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    s_inv[j] = __ldg(inv + (size_t)t * k + j);
+    s_w[j] = __ldg(w + (size_t)t * k + j);
+  }
+  __syncthreads();
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    float acc[8];
+    if (ys) {
+      const float4 a = __ldg((const float4*)(ys + (size_t)t * d + c));
+      const float4 b = __ldg((const float4*)(ys + (size_t)t * d + c + 4));
+      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    }
+    for (int j = 0; j < k; ++j) {
+      const int p = s_inv[j];
+      if (p < 0) continue;
+      const uint4 v = __ldg((const uint4*)(O + (size_t)p * d + c));
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      const float wj = s_w[j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(wj, __uint_as_float(wv[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      o[i] = *(const uint32_t*)&p2;
+    }
+    *(uint4*)(y + (size_t)t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ---------------------------------------------------------------- weight packing (setup)
+// fp32 rows [R][K] -> E2M1 codes (2 per byte, element 2j in the low nibble) at packed row
+// dst_row(r), and E8M0 scales into the MMA scale-factor atom layout
+// [m_tiles][K/128][2][512]: row rr of a 256-row tile, K-block kb ->
+//   ((mt * (K/128) + kb/4) * 2 + half) * 512 + (rr%32)*16 + ((rr%128)/32)*4 + kb%4.
+// interleave != 0: rows of two sources (gate, up) go to packed rows
+//   256*(r/128) + 128*src + r%128.
+__global__ void pack_mxfp4_kernel(const float* __restrict__ src0, const float* __restrict__ src1,
+                                  int R, int K, int interleave, uint8_t* __restrict__ wdst,
+                                  uint8_t* __restrict__ sdst) {
+  const int nb = K >> 5;
+  const int nsrc = interleave ? 2 : 1;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)nsrc * R * nb) return;
+  const int which = (int)(gid / ((long long)R * nb));
+  const long long rem = gid - (long long)which * R * nb;
+  const int r = (int)(rem / nb);
+  const int b = (int)(rem - (long long)r * nb);
+  const float* src = which ? src1 : src0;
+  const float4* p = (const float4*)(src + (size_t)r * K + b * 32);
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = __ldg(p + i);
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = mx_scale_exp(amax, 2);
+  const float s = pow2_neg(e);
+  uint32_t wds[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc |= cvt_e2m1x2(v[8 * i + 2 * j] * s, v[8 * i + 2 * j + 1] * s) << (8 * j);
+    wds[i] = acc;
+  }
+  const int pr = interleave ? 256 * (r >> 7) + 128 * which + (r & 127) : r;
+  *(uint4*)(wdst + (size_t)pr * (K / 2) + b * 16) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  const int mt = pr >> 8, half = (pr >> 7) & 1, rr = pr & 127;
+  const size_t so = ((size_t)(mt * (K >> 7) + (b >> 2)) * 2 + half) * 512 + (rr & 31) * 16 +
+                    (rr >> 5) * 4 + (b & 3);
+  sdst[so] = (uint8_t)(e + 127);
+}
+
+// Router weights W_r fp32 [d][E] -> three bf16 planes W^T [E][3d] with
+// W = hi + mid + lo exactly (hi = bf16(W), mid = bf16(W - hi), lo = bf16(W - hi - mid)).
+__global__ void router_split_kernel(const float* __restrict__ W, int d, int E,
+                                    __nv_bfloat16* __restrict__ planes) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int i = i0 + r, e = e0 + threadIdx.x;
+    tile[r][threadIdx.x] = (i < d && e < E) ? W[(size_t)i * E + e] : 0.0f;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int e = e0 + r, i = i0 + threadIdx.x;
+    if (e < E && i < d) {
+      const float w = tile[threadIdx.x][r];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+      const float r1 = w - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(mid);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+      __nv_bfloat16* row = planes + (size_t)e * 3 * d;
+      row[i] = hi;
+      row[d + i] = mid;
+      row[2 * d + i] = lo;
+    }
+  }
+}
+
+}  // namespace moe

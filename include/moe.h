@@ -1,0 +1,171 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) Kimi-K3 MoE feed-forward layer.
+ *
+ * The layer (what the source pages fix):
+ *   - "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, rows "Sigmoid router
+ *     with Quantile Balancing", "Stable LatentMoE routed experts (SiTU-GLU)" and
+ *     "Shared expert": sigmoid scores pick 16 of 896 GLU experts per token; one always-on,
+ *     ungated bf16 shared expert reads the same input; the block diagram adds the two.
+ *   - "Kimi K3" (llm-atlas), raw config fields: hidden_size 7168, num_experts 896,
+ *     num_experts_per_token 16, moe_intermediate_size 3072, moe_renormalize true,
+ *     routed_scaling_factor 1; Key facts, Dtype row: experts MXFP4, shared expert high
+ *     precision.
+ *   - "Kimi K3, previewed" (embedl blog), specifications figure caption: MXFP4 weights,
+ *     MXFP8 activations.
+ * Readings where the pages are silent: the GLU activation is SiLU (the SiTU formula is
+ * unpublished), experts act on d_model directly, the router bias is added to the logit,
+ * ties in top-k go to the lower expert index, the GLU output is requantised to MXFP8
+ * before the down projection.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller; the library
+ *     never frees them.  "host" pointers are ordinary CPU memory.
+ *   - Matrices are row-major.  Weights are stored out x in (row = output channel).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *     default stream); none synchronises the host except moe_plan_check and
+ *     moe_debug_read_status.
+ *   - Errors are returned as moe_status_t; nothing is thrown.  Argument checks happen
+ *     before any launch, so an error return leaves outputs untouched.
+ *   - Device-side faults (an out-of-range expert id, a pipeline wait that timed out) are
+ *     OR-ed into the plan's status word; moe_plan_check reads and clears it.
+ */
+#ifndef MOE_SM100_H
+#define MOE_SM100_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_plan_s* moe_plan_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum value */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* d, I, I_shared not multiples of 128; k > 32; T > T_max */
+  MOE_ERR_ALIGNMENT = 3,         /* a pointer below its required alignment */
+  MOE_ERR_CUDA = 4,              /* a CUDA runtime / driver call or launch failed */
+  MOE_ERR_TIMEOUT = 5,           /* a kernel gave up on a bounded wait (moe_plan_check) */
+  MOE_ERR_NOT_INITIALIZED = 6,   /* no workspace attached to the plan */
+  MOE_ERR_DEVICE_FAULT = 7       /* a kernel flagged bad input (e.g. expert id >= E) */
+} moe_status_t;
+
+typedef enum { MOE_ACT_SILU_GLU = 0 } moe_act_t;
+typedef enum { MOE_BIAS_LOGIT = 0 } moe_bias_mode_t;
+
+/* Packed MXFP4 expert weights (device pointers, all 256-byte aligned).
+ *   w_gu: E2M1 codes of gate and up, [E][2I][d/2] bytes, element 2j of a row in the low
+ *         nibble of byte j.  Rows are channel blocks of 128 interleaved as
+ *         gate[0:128], up[0:128], gate[128:256], up[128:256], ...
+ *   s_gu: E8M0 scales (one per 32 elements along d) in the tensor-core scale-factor
+ *         tiling [E][2I/256][d/128][2][512] (see moe_pack_expert_mxfp4).
+ *   w_dn: E2M1 codes of down, [E][d][I/2] bytes.
+ *   s_dn: E8M0 scales of down, [E][ceil(d/256)][I/128][2][512].
+ * Sizes come from moe_expert_bytes; contents from moe_pack_expert_mxfp4. */
+typedef struct {
+  void* w_gu;
+  void* s_gu;
+  void* w_dn;
+  void* s_dn;
+} moe_experts_mxfp4;
+
+/* bf16 shared expert (device pointers, 16-byte aligned).
+ *   w_gu: [2 I_s][d], gate/up interleaved in 128-row blocks as above.
+ *   w_dn: [d][I_s]. */
+typedef struct {
+  void* w_gu;
+  void* w_dn;
+} moe_shared_bf16;
+
+/* ---- plan ---------------------------------------------------------------------------
+ * moe_plan_create: checks the layer shape and the device, allocates nothing on the
+ * device.  T_max bounds the tokens of any later call; d, I, I_shared multiples of 128
+ * (I_shared = 0: no shared expert); 1 <= k <= min(E, 32); E <= 4096.
+ * Returns the plan in *out (host object, freed by moe_plan_destroy). */
+moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared,
+                             moe_act_t act, moe_bias_mode_t bias_mode, int flags,
+                             moe_plan_t* out);
+/* Device workspace the plan needs for T_max tokens, in bytes (host output). */
+moe_status_t moe_plan_workspace_bytes(moe_plan_t plan, size_t* bytes);
+/* Attach caller-owned device workspace (256-byte aligned, >= moe_plan_workspace_bytes).
+ * The plan borrows it until destroyed or given another one. */
+moe_status_t moe_plan_set_workspace(moe_plan_t plan, void* dev_ptr, size_t bytes);
+/* Synchronises `stream`, returns MOE_ERR_TIMEOUT / MOE_ERR_DEVICE_FAULT if a kernel since
+ * the last check flagged one (bit values in *device_bits, may be NULL), and clears it. */
+moe_status_t moe_plan_check(moe_plan_t plan, void* stream, unsigned int* device_bits);
+moe_status_t moe_plan_destroy(moe_plan_t plan);
+const char* moe_status_string(moe_status_t s);
+
+/* ---- a1: MXFP8 activation quantiser ------------------------------------------------
+ * OCP MX rule per 32-element block along a row: scale byte = floor(log2 amax) - 8 + 127
+ * (clamped to [0, 254]; all-zero block -> 0), element = E4M3 round-to-nearest-even of
+ * v / 2^(scale-127), saturating to +-448, sign kept.
+ * x_bf16: device [rows][cols] bf16; q_e4m3: device [rows][cols]; scale_e8m0: device
+ * [rows][cols/32].  cols % 32 == 0; x 16-byte aligned, q 16-byte aligned. */
+moe_status_t moe_quant_mxfp8(const void* x_bf16, int rows, int cols, uint8_t* q_e4m3,
+                             uint8_t* scale_e8m0, void* stream);
+
+/* ---- a2/a3: router --------------------------------------------------------------------
+ * z = x . W_r + bias (fp32-accurate: W_r is split into three bf16 terms on the tensor
+ * cores), s = sigmoid(z); per token the k largest z in descending order (lower expert
+ * index on ties) and w_j = s_j / sum of the selected s.
+ * x_bf16: device [T][d]; W_r: device fp32 [d][E]; bias: device fp32 [E] or NULL;
+ * idx: device int32 [T][k]; w: device fp32 [T][k]; logits_opt: device fp32 [T][E] or
+ * NULL (receives z).  Uses the plan workspace. */
+moe_status_t moe_route(moe_plan_t plan, const void* x_bf16, int T, const float* W_r,
+                       const float* bias, int32_t* idx, float* w, float* logits_opt,
+                       void* stream);
+
+/* ---- a4: grouping by expert -----------------------------------------------------------
+ * counts[e] = assignments to expert e; offsets = exclusive prefix sum (offsets[E] = T*k);
+ * perm_tok[p] = token of the p-th assignment in (expert, token) order; inv[t][j] = the
+ * position of assignment (t, j).  idx: device int32 [T][k] with distinct ids per token.
+ * Outputs are device int32 arrays of E, E+1, T*k, T*k entries.  Ids outside [0, E) are
+ * skipped and flagged (MOE_ERR_DEVICE_FAULT at moe_plan_check). */
+moe_status_t moe_permute(moe_plan_t plan, const int32_t* idx, int T, int32_t* counts,
+                         int32_t* offsets, int32_t* perm_tok, int32_t* inv, void* stream);
+
+/* ---- a4..a9: the layer ----------------------------------------------------------------
+ * y = bf16( shared(x) + sum_j w[t][j] * expert_{idx[t][j]}(x) ), where an expert is
+ * down(silu(x Wg^T) * (x Wu^T)) on MXFP8 x and MXFP4 weights, its GLU output requantised
+ * to MXFP8, and shared(x) = bf16(silu(x Wsg^T) * (x Wsu^T)) Wsd^T in bf16/fp32.
+ * x_bf16: device [T][d]; idx/w: device [T][k] (e.g. from moe_route); experts: packed
+ * weights; shared: NULL when the plan has I_shared = 0; y_bf16: device [T][d].
+ * T = 0 is a no-op.  Uses the plan workspace (one call at a time per plan). */
+moe_status_t moe_forward(moe_plan_t plan, const void* x_bf16, int T, const int32_t* idx,
+                         const float* w, const moe_experts_mxfp4* experts,
+                         const moe_shared_bf16* shared, void* y_bf16, void* stream);
+
+/* ---- setup helpers (not on the timed path) --------------------------------------------
+ * Byte sizes of the four packed expert arrays for E experts (host outputs). */
+moe_status_t moe_expert_bytes(int d, int I, int E, size_t* w_gu, size_t* s_gu, size_t* w_dn,
+                              size_t* s_dn);
+/* MXFP4-quantise expert e's fp32 masters (device: w_gate, w_up [I][d], w_down [d][I];
+ * blocks of 32 along the input dimension, same MX rule as above with E2M1 elements,
+ * max 6, emax 2) into the packed arrays of `dst`. */
+moe_status_t moe_pack_expert_mxfp4(int d, int I, int e, const float* w_gate, const float* w_up,
+                                   const float* w_down, const moe_experts_mxfp4* dst,
+                                   void* stream);
+/* Lay out the bf16 shared expert (device: w_gate, w_up [I_s][d], w_down [d][I_s]) into
+ * dst (device buffers of 2*I_s*d and d*I_s bf16). */
+moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const void* w_up,
+                                  const void* w_down, const moe_shared_bf16* dst, void* stream);
+
+/* ---- introspection (tests) ----------------------------------------------------------
+ * Device pointer and size of a workspace buffer after a call, for checking the steps:
+ *   0 xq  E4M3 [T*k][d] activations in expert order
+ *   1 xs  u32 scale words [d/128][T*k] (byte j = 32-block 4m+j of a row)
+ *   2 hq  E4M3 [T*k][I] GLU output in expert order
+ *   3 hs  u32 scale words [I/128][T*k]
+ *   4 O   bf16 [T*k][d] expert outputs in expert order
+ *   5 ys  fp32 [T][d] shared expert output
+ *   6 logits fp32 [T][E]
+ * Row counts use the T of the last call. */
+moe_status_t moe_debug_buffer(moe_plan_t plan, int which, void** dev_ptr, size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_SM100_H */

@@ -1,0 +1,58 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every entry point that
+include/moe.h declares (no compute calls: this runs without a GPU)."""
+import ctypes
+import os
+import re
+
+from block_scaled_moe_sigmoid_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moe_plan_create", "moe_route", "moe_forward", "moe_quant_mxfp8", "moe_permute"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    path = build.build()
+    L = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(declared_functions()) == set(api.SIGNATURES)
+
+
+def test_host_side_argument_checks_without_gpu():
+    L = api.lib()
+    h = ctypes.c_void_p()
+    # bad shapes are rejected before anything touches a device
+    assert L.moe_plan_create(16, 100, 8, 2, 128, 0, 0, 0, 0, ctypes.byref(h)) == 2
+    assert L.moe_plan_create(16, 128, 8, 33, 128, 0, 0, 0, 0, ctypes.byref(h)) == 2
+    assert L.moe_plan_create(16, 128, 8, 9, 128, 0, 0, 0, 0, ctypes.byref(h)) == 2
+    assert L.moe_plan_create(-1, 128, 8, 2, 128, 0, 0, 0, 0, ctypes.byref(h)) == 1
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 1, 0, 0, ctypes.byref(h)) == 1
+    assert L.moe_quant_mxfp8(None, 4, 33, None, None, None) == 2
+    assert L.moe_status_string(3) == b"misaligned pointer"
+    sizes = api.moe_expert_bytes(7168, 3072, 896)
+    # 896 experts x 3 matrices x 7168 x 3072 x (0.5 + 1/32) bytes
+    assert sum(sizes) == 896 * 3 * 7168 * 3072 * 17 // 32
+
+
+def test_workspace_size_grows_with_tokens():
+    L = api.lib()
+    h1, h2 = ctypes.c_void_p(), ctypes.c_void_p()
+    assert L.moe_plan_create(64, 7168, 896, 16, 3072, 3072, 0, 0, 0, ctypes.byref(h1)) == 0
+    assert L.moe_plan_create(8192, 7168, 896, 16, 3072, 3072, 0, 0, 0, ctypes.byref(h2)) == 0
+    n1, n2 = ctypes.c_size_t(), ctypes.c_size_t()
+    L.moe_plan_workspace_bytes(h1, ctypes.byref(n1))
+    L.moe_plan_workspace_bytes(h2, ctypes.byref(n2))
+    assert 0 < n1.value < n2.value < 8 << 30
+    L.moe_plan_destroy(h1)
+    L.moe_plan_destroy(h2)

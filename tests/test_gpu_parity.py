@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bit-exact: MXFP8 quantised bytes and scales, packed MXFP4 weights, routing indices
+given identical logits, the permutation.  Within tolerance: logits, routing weights, the
+layer output (max relative error <= 2e-2, mean <= 2e-3 over tokens whose k/k+1 score
+gap is >= 1e-6; the others are counted)."""
+import numpy as np
+import pytest
+import torch
+
+from block_scaled_moe_sigmoid_b200 import api, synth
+from oracle import layer, mx, permute as operm, router
+
+from .gpu_helpers import Case, layer_stats, unpack_expert_codes
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL, MEAN_REL = 2e-2, 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    api.lib()
+
+
+# ------------------------------------------------------------------ a1: MXFP8 quantiser
+def _quant_inputs():
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(37, 224, generator=g) * torch.logspace(-30, 30, 224).float()  # ragged rows, wide range
+    x[0] = 0.0
+    x[1, :32] = -0.0
+    x[2, :32] = 448.0 * 2.0 ** 10
+    x[3, :32] *= 1e-38                 # a block of bf16 subnormals and zeros
+    x[3, 5] = float(2.0 ** -133)
+    x[4, :32] = torch.tensor([17.0, 19.0, -17.0, 480.0] * 8)
+    return x.to(torch.bfloat16)
+
+
+def test_quant_mxfp8_bit_exact():
+    x = _quant_inputs()
+    q, s = api.moe_quant_mxfp8(x.cuda())
+    q_ref, s_ref = mx.quantize_mx(x.float().numpy().astype(np.float64), "e4m3")
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quant_mxfp8_toy_and_empty():
+    wl = synth.WORKLOADS["toy"]
+    x = synth.draw_x(wl)
+    q, s = api.moe_quant_mxfp8(x.cuda())
+    q_ref, s_ref = mx.quantize_mx(x.float().numpy().astype(np.float64), "e4m3")
+    assert np.array_equal(q.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
+    q0, s0 = api.moe_quant_mxfp8(torch.empty((0, 64), dtype=torch.bfloat16, device="cuda"))
+    assert q0.shape == (0, 64)
+
+
+# ------------------------------------------------------------------ a0: MXFP4 packing
+def test_pack_mxfp4_bit_exact():
+    wl = synth.custom(seed=5, d=384, I=256, E=3)
+    ex = api.Experts(wl.d, wl.I, wl.E)
+    for e in range(wl.E):
+        ms = synth.draw_expert(wl, e)
+        ex.pack(e, *(t.cuda() for t in ms))
+        torch.cuda.synchronize()
+        got = unpack_expert_codes(ex, e, wl.d, wl.I)
+        ref = layer.quantize_expert(*(t.numpy() for t in ms))
+        for name in ("gate", "up", "down"):
+            assert np.array_equal(got[name][1], ref[name][1]), (e, name, "scales")
+            assert np.array_equal(got[name][0], ref[name][0]), (e, name, "codes")
+
+
+# ------------------------------------------------------------------ a4: permutation
+@pytest.mark.parametrize("T,E,k", [(128, 32, 4), (1, 8, 2), (1000, 896, 16), (513, 5, 5)])
+def test_permute_bit_exact(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    plan = api.Plan(T, 128, E, k, 128)
+    counts, offsets, perm_tok, inv = plan.permute(idx.cuda())
+    c_ref, o_ref, p_ref, i_ref = operm.permute(idx.numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), c_ref)
+    assert np.array_equal(offsets.cpu().numpy(), o_ref)
+    assert np.array_equal(perm_tok.cpu().numpy(), p_ref)
+    assert np.array_equal(inv.cpu().numpy(), i_ref)
+    assert plan.check()[0] == 0
+
+
+def test_permute_flags_bad_ids():
+    plan = api.Plan(4, 128, 8, 2, 128)
+    idx = torch.tensor([[0, 1], [2, 9], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")
+    _, _, _, inv = plan.permute(idx)
+    code, bits = plan.check()
+    assert code == 7 and bits & 2
+    assert inv[1, 1].item() == -1
+
+
+# ------------------------------------------------------------------ a2/a3: router
+def _check_route(case, atol_z=2e-5):
+    T, E, k = case.T, case.wl.E, case.wl.k
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    idx, w = case.plan.route(case.x, case.W_r, case.bias, logits=logits)
+    torch.cuda.synchronize()
+    z_gpu = logits.cpu().numpy().astype(np.float64)
+    z_ref, (idx_o, w_o, gap) = case.oracle_route()
+    assert np.max(np.abs(z_gpu - z_ref)) < atol_z
+    # bit-exact selection given identical scores
+    idx_g, w_g, _ = router.route(z_gpu, k)
+    assert np.array_equal(idx.cpu().numpy(), idx_g)
+    assert np.allclose(w.cpu().numpy(), w_g, rtol=2e-6, atol=1e-7)
+    # against the oracle's own fp64 routing, mismatches only on near ties
+    mism = np.any(idx.cpu().numpy() != idx_o, axis=1)
+    assert not np.any(mism & (gap >= 1e-6))
+    return idx, w, idx_o, w_o, gap
+
+
+def test_route_toy():
+    case = Case(synth.WORKLOADS["toy"])
+    _check_route(case)
+
+
+def test_route_ragged_and_biased():
+    wl = synth.custom(seed=3, T=333, d=256, E=40, k=7, I=128)
+    bias = -2.4 * torch.log(torch.randperm(40, generator=torch.Generator().manual_seed(1)).double() + 1)
+    case = Case(wl, bias=bias)
+    _check_route(case)
+
+
+# ------------------------------------------------------------------ the layer
+def _check_layer(case, tokens=None, stage_checks=False):
+    idx, w, idx_o, w_o, gap = _check_route(case)
+    y = case.plan.forward(case.x, idx, w, case.experts, case.shared)
+    assert case.plan.check()[0] == 0
+    y = y.float().cpu().numpy().astype(np.float64)
+    x = case.x_np()
+    rows = np.arange(case.T) if tokens is None else np.asarray(tokens)
+    y_ref = layer.moe_layer(x, idx_o, w_o, case.oracle_expert, case.oracle_shared(), tokens=rows)
+    st = layer_stats(y[rows], y_ref, gap[rows])
+    assert st["max_rel"] <= MAX_REL and st["mean_rel"] <= MEAN_REL, st
+    if stage_checks:
+        _stage_checks(case, idx.cpu().numpy(), w.cpu().numpy())
+    return st
+
+
+def _stage_checks(case, idx, w):
+    """Intermediates in expert order against the oracle on the same routing."""
+    wl, T = case.wl, case.T
+    A = T * wl.k
+    _, offs, perm_tok, inv = operm.permute(idx, wl.E)
+    x = case.x_np()
+    xq_ref, xs_ref = mx.quantize_mx(x, "e4m3")
+    xq = case.plan.debug_tensor(0, torch.uint8, (A, wl.d)).cpu().numpy()
+    xs = case.plan.debug_tensor(1, torch.int32, (wl.d // 128, A)).cpu().numpy().view(np.uint8)
+    xs = xs.reshape(wl.d // 128, A, 4).transpose(1, 0, 2).reshape(A, wl.d // 32)
+    assert np.array_equal(xq, xq_ref[perm_tok])
+    assert np.array_equal(xs, xs_ref[perm_tok])
+    # GLU output (MXFP8): decoded values agree up to one E4M3 step where fp32 and fp64
+    # land on different sides of a rounding boundary
+    hq = case.plan.debug_tensor(2, torch.uint8, (A, wl.I)).cpu().numpy()
+    hs = case.plan.debug_tensor(3, torch.int32, (wl.I // 128, A)).cpu().numpy().view(np.uint8)
+    hs = hs.reshape(wl.I // 128, A, 4).transpose(1, 0, 2).reshape(A, wl.I // 32)
+    H = mx.dequantize_mx(hq, hs, "e4m3")
+    X = mx.dequantize_mx(xq_ref, xs_ref, "e4m3")
+    worst, mism = 0.0, 0
+    O = case.plan.debug_tensor(4, torch.bfloat16, (A, wl.d)).float().cpu().numpy()
+    for e in range(wl.E):
+        rows = np.arange(offs[e], offs[e + 1])
+        if len(rows) == 0:
+            continue
+        Wg, Wu, Wd = case.oracle_expert(e)
+        o_ref, a_ref, hq_ref, hs_ref = layer.expert_forward(X[perm_tok[rows]], Wg, Wu, Wd)
+        H_ref = mx.dequantize_mx(hq_ref, hs_ref, "e4m3")
+        diff = np.abs(H[rows] - H_ref)
+        scale = np.repeat(mx.e8m0_value(hs_ref), 32, axis=1)
+        mism += int(np.sum(diff > 0))
+        worst = max(worst, float(np.max(diff / (np.abs(H_ref) + scale * 2.0 ** -9))))
+        # expert outputs (bf16, expert order) against the oracle's, row-normwise
+        rel = np.linalg.norm(O[rows] - o_ref, axis=1) / np.linalg.norm(o_ref, axis=1)
+        assert rel.max() < 1e-2, (e, rel.max())
+    assert worst <= 0.13, worst                      # at most one E4M3 step (2^-3 relative)
+    assert mism <= 0.01 * A * wl.I, mism
+
+
+def test_layer_toy():
+    case = Case(synth.WORKLOADS["toy"])
+    st = _check_layer(case, stage_checks=True)
+    print("toy", st)
+
+
+def test_layer_with_shared_ragged():
+    wl = synth.custom(seed=7, T=203, d=384, E=12, k=3, I=256, I_shared=384)
+    case = Case(wl)
+    _check_layer(case, stage_checks=True)
+
+
+def test_layer_single_token_and_empty_experts():
+    wl = synth.custom(seed=8, T=1, d=256, E=64, k=4, I=128)
+    case = Case(wl)
+    _check_layer(case)
+
+
+def test_layer_hot_experts_span_several_tiles():
+    """A bias sends every token to the same experts: each carries T=400 rows, which the
+    GEMMs split over 3 tiles of <= 160 rows."""
+    wl = synth.custom(seed=9, T=400, d=256, E=16, k=4, I=128, I_shared=128)
+    bias = torch.zeros(16)
+    bias[[3, 7, 11, 12]] = 40.0
+    case = Case(wl, bias=bias)
+    _check_layer(case, stage_checks=True)
+
+
+def test_layer_dense_mixture_k_equals_e():
+    wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
+    case = Case(wl)
+    _check_layer(case)
+
+
+def test_forward_t0_is_noop():
+    wl = synth.custom(seed=1, T=4, d=128, E=4, k=2, I=128)
+    case = Case(wl)
+    y = torch.full((0, 128), 1.0, dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((0, 2), dtype=torch.int32, device="cuda")
+    w = torch.zeros((0, 2), dtype=torch.float32, device="cuda")
+    case.plan.forward(y, idx, w, case.experts, None, y=y)
+
+
+def test_forward_rejects_bad_arguments():
+    wl = synth.custom(seed=1, T=4, d=128, E=4, k=2, I=128)
+    case = Case(wl)
+    idx = torch.zeros((4, 2), dtype=torch.int32, device="cuda")
+    w = torch.zeros((4, 2), dtype=torch.float32, device="cuda")
+    with pytest.raises(api.MoeError) as e:        # T > T_max
+        big = torch.zeros((8, 128), dtype=torch.bfloat16, device="cuda")
+        case.plan.forward(big, torch.zeros((8, 2), dtype=torch.int32, device="cuda"),
+                          torch.zeros((8, 2), device="cuda"), case.experts)
+    assert e.value.code == 2
+    with pytest.raises(api.MoeError) as e:        # misaligned x
+        raw = torch.zeros(4 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+        case.plan.forward(raw[1:1 + 512].view(4, 128), idx, w, case.experts)
+    assert e.value.code == 3
