@@ -1,0 +1,362 @@
+"""Benchmark of the Kimi-K3 MoE feed-forward layer on B200.
+
+One step = the whole hot path on one batch: moe_route (router GEMM, sigmoid top-k) and
+moe_forward (grouping, MXFP8 quantise, gate/up grouped GEMM + GLU + requant, down grouped
+GEMM, shared expert, combine), inputs resident in HBM.  Default workload: Kimi-K3 prefill,
+T=8192 tokens, d=7168, 896 experts, top-16, I=3072, one bf16 shared expert (I=3072).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: token batches are independent, so N ranks run N replicas of the workload
+(weak scaling, no collective on the data path); the timing is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload
+(rank 0 only) and extrapolates to the full batch.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at K3 shape (T=8192); % FP4 tensor peak, decode % HBM BW"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="k3_prefill_t8192")
+    ap.add_argument("--T", type=int, default=None, help="override the token count")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- oracle timing (CPU)
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_seconds(wl, T, x_dev, W_r_dev, bias_dev, n_router, n_experts, n_shared, seed=0):
+    """Time the fp64 oracle on a bounded sample and extrapolate to the full batch of T tokens:
+    router logits + top-k for n_router tokens (scaled by T / n_router), n_experts experts
+    each with the mean load T*k/E rows (scaled by E / n_experts; includes quantising and
+    decoding the expert's MXFP4 weights), and the shared expert on n_shared tokens
+    (scaled by T / n_shared).  Returns (seconds for T tokens, sample description)."""
+    import numpy as np
+    import torch
+
+    from block_scaled_moe_sigmoid_b200 import synth
+    from oracle import layer, mx, router
+
+    g = np.random.default_rng(seed)
+    rows = np.sort(g.choice(T, size=min(n_router, T), replace=False))
+    x = x_dev.float().cpu().numpy().astype(np.float64)
+    W_r = W_r_dev.cpu().numpy()
+    b = bias_dev.cpu().numpy()
+    t0 = time.perf_counter()
+    z = router.router_logits(x[rows], W_r, b)
+    router.route(z, wl.k)
+    t_router = (time.perf_counter() - t0) * T / len(rows)
+
+    load = max(1, int(round(T * wl.k / wl.E)))
+    t_exp = 0.0
+    for i in range(n_experts):
+        e = int(g.integers(wl.E))
+        masters = [t.cpu().numpy() for t in synth.draw_expert(wl, e, device=x_dev.device.type)]
+        tok = g.choice(T, size=load, replace=True)
+        t0 = time.perf_counter()
+        Wg, Wu, Wd = layer.decode_expert(layer.quantize_expert(*masters))
+        xq, xs = mx.quantize_mx(x[tok], "e4m3")
+        layer.expert_forward(mx.dequantize_mx(xq, xs, "e4m3"), Wg, Wu, Wd)
+        t_exp += time.perf_counter() - t0
+    t_exp *= wl.E / max(n_experts, 1)
+
+    t_sh = 0.0
+    if wl.I_shared:
+        sw = tuple(t.float().cpu().numpy().astype(np.float64)
+                   for t in synth.draw_shared(wl, device=x_dev.device.type))
+        srows = rows[:min(n_shared, len(rows))]
+        t0 = time.perf_counter()
+        layer.shared_expert(x[srows], *sw)
+        t_sh = (time.perf_counter() - t0) * T / len(srows)
+    desc = (f"router on {len(rows)} of {T} tokens, {n_experts} of {wl.E} experts at the mean "
+            f"load of {load} rows (weights quantised+decoded per expert), shared expert on "
+            f"{min(n_shared, len(rows))} tokens; each part scaled linearly to T={T}")
+    return t_router + t_exp + t_sh, desc
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        load = [s for s in sms if mx and s > 0.3 * mx] or sms
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ---------------------------------------------------------------- our arm
+def setup(wl, T, device):
+    import torch
+
+    from block_scaled_moe_sigmoid_b200 import api, synth
+    x = synth.draw_x(wl, T, device=device)
+    W_r, bias = synth.draw_router(wl, device=device)
+    plan = api.Plan(T, wl.d, wl.E, wl.k, wl.I, wl.I_shared, device=device)
+    ex = api.Experts(wl.d, wl.I, wl.E, device=device)
+    for e in range(wl.E):
+        g, u, dn = synth.draw_expert(wl, e, device=device)
+        ex.pack(e, g, u, dn)
+        del g, u, dn
+    sh = None
+    if wl.I_shared:
+        sh = api.Shared(wl.d, wl.I_shared, device=device)
+        sh.pack(*synth.draw_shared(wl, device=device))
+    torch.cuda.synchronize()
+    return x, W_r, bias, plan, ex, sh
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from block_scaled_moe_sigmoid_b200 import api, synth
+    wl = synth.WORKLOADS[args.workload]
+    T = args.T or (wl.sweep[-1] if wl.sweep else wl.T)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    x, W_r, bias, plan, ex, sh = setup(wl, T, "cuda")
+    idx = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, wl.k), dtype=torch.float32, device=dev)
+    y = torch.empty((T, wl.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        api.moe_route(plan.handle, x, W_r, bias, wl.k, idx=idx, w=w)
+        api.moe_forward(plan.handle, x, idx, w, ex, sh, y)
+
+    for _ in range(args.warmup):
+        one_step()
+    code, bits = plan.check()
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits} after warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    api.moe_plan_set_profiling(plan.handle, True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    stages = api.moe_plan_stage_ms(plan.handle)
+    api.moe_plan_set_profiling(plan.handle, False)
+    clk = clocks.stop()
+    code, bits = plan.check()
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits} in the timed region")
+    launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(x)
+        for _ in range(max(1, args.warmup)):
+            x_dev.copy_(x_host, non_blocking=True)
+            api.moe_route(plan.handle, x_dev, W_r, bias, wl.k, idx=idx, w=w)
+            api.moe_forward(plan.handle, x_dev, idx, w, ex, sh, y)
+            y_host.copy_(y, non_blocking=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            x_dev.copy_(x_host, non_blocking=True)
+            api.moe_route(plan.handle, x_dev, W_r, bias, wl.k, idx=idx, w=w)
+            api.moe_forward(plan.handle, x_dev, idx, w, ex, sh, y)
+            y_host.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * T * args.steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": x.numel() * x.element_size(),
+               "d2h_bytes_per_step": y.numel() * y.element_size()}
+
+    # ---- roofline of the dominant kernel (routed gate/up GEMM)
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    gu_ms, gu_n = stages["gate_up_glu"]
+    A = T * wl.k
+    flops = 2.0 * A * wl.d * (2 * wl.I)
+    if peaks.get("bf16_tflops_sustained"):
+        peak, peak_src = 2.0 * peaks["bf16_tflops_sustained"], "measured"
+    else:
+        peak, peak_src = 2.0 * 1400.0, "fallback"
+    achieved = flops / (gu_ms / gu_n / 1e3) / 1e12 if gu_n else None
+    roofline = {"kernel": "gemm_kernel<KIND_MX, EPI_GLU_MX8> (routed gate/up + SiLU-GLU + MXFP8 requant)",
+                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak if achieved else None, "traffic": None,
+                "peak_note": f"FP8-rate tensor pipe = 2 x {peak_src} sustained bf16 GEMM "
+                             f"(kind::mxf8f6f4 issues at the FP8 rate)",
+                "ms_per_launch": gu_ms / gu_n if gu_n else None,
+                "flops_per_launch": flops}
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    w_bytes = wl.E * 3 * wl.d * wl.I * 17 / 32
+    stage_ms = {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()}
+
+    out = None
+    if rank == 0:
+        value = world * T * args.steps / (ms / 1e3)
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4xmxfp8 (fp32 acc); bf16 shared/router",
+            "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights, random-init)",
+            "config": {"workload": args.workload, "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I,
+                       "I_shared": wl.I_shared, "seed": wl.seed, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2: every step streams "
+                             f"{w_bytes / 1e9:.1f} GB of expert weights"},
+            "roofline": roofline,
+            "hbm_view": {"weight_bytes_per_step": w_bytes,
+                         "achieved_gbs": w_bytes / (ms / args.steps / 1e3) / 1e9,
+                         "peak_gbs": hbm},
+            "stage_ms_per_launch": stage_ms,
+            "clocks": clk, "e2e": e2e, "gpu_launches": launches,
+        }
+    return out, (x, W_r, bias, wl, T)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    out, data = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        x, W_r, bias, wl, T = data
+        secs, desc = oracle_sample_seconds(wl, T, x, W_r, bias, n_router=256, n_experts=2, n_shared=64)
+        out["cpu_baseline"] = {"value": T / secs, "unit": UNIT, "cores": blas_threads(),
+                               "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import torch
+
+    from block_scaled_moe_sigmoid_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    T = args.T or (wl.sweep[-1] if wl.sweep else wl.T)
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
+    x = synth.draw_x(wl, T, device=gen)
+    W_r, bias = synth.draw_router(wl, device=gen)
+    secs = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        s, desc = oracle_sample_seconds(wl, T, x, W_r, bias, n_router=32, n_experts=1, n_shared=8, seed=i)
+        if i >= args.warmup:
+            secs.append(s)
+    total = sum(secs)
+    value = T * len(secs) / total
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * total / len(secs), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+           "data": "synthetic (seeded)",
+           "config": {"workload": args.workload, "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I,
+                      "I_shared": wl.I_shared, "seed": wl.seed},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

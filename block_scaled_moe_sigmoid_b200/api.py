@@ -35,7 +35,15 @@ SIGNATURES = {
     "moe_pack_expert_mxfp4": [_I, _I, _I, _P, _P, _P, _P, _P],
     "moe_pack_shared_bf16": [_I, _I, _P, _P, _P, _P, _P],
     "moe_debug_buffer": [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_S)],
+    "moe_plan_set_profiling": [_P, _I],
+    "moe_plan_set_option": [_P, _I, _I],
+    "moe_plan_stage_ms": [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _I],
 }
+
+STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "gate_up_glu",
+          "down", "shared_gate_up", "shared_down", "combine"]
+# kernel launches per recorded stage instance
+STAGE_KERNELS = {"permute": 3}
 
 
 class MoeError(RuntimeError):
@@ -176,6 +184,26 @@ def moe_debug_buffer(plan, which):
     p, n = ctypes.c_void_p(), ctypes.c_size_t()
     _call("moe_debug_buffer", plan, which, ctypes.byref(p), ctypes.byref(n))
     return p.value, n.value
+
+
+MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B = 0, 1
+
+
+def moe_plan_set_option(plan, option, value):
+    _call("moe_plan_set_option", plan, option, int(value))
+
+
+def moe_plan_set_profiling(plan, enable=True):
+    _call("moe_plan_set_profiling", plan, 1 if enable else 0)
+
+
+def moe_plan_stage_ms(plan):
+    """{stage: (summed ms, recorded launches)} since profiling was enabled / last queried."""
+    n = len(STAGES)
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_int * n)()
+    _call("moe_plan_stage_ms", plan, ms, cnt, n)
+    return {STAGES[i]: (ms[i], cnt[i]) for i in range(n)}
 
 
 # ------------------------------------------------------------------ buffers

@@ -4,10 +4,12 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/moe.h"
 #include "gemm.cuh"
 #include "kernels.cuh"
+#include "router.cuh"
 
 using namespace moe;
 
@@ -16,6 +18,8 @@ namespace {
 constexpr int kBN = 160;      // tokens per GEMM tile (MMA N <= 160)
 constexpr int kStages = 4;    // smem pipeline depth of every GEMM
 constexpr int kPermThreads = 256;
+constexpr int kRouterBN = 128;  // tokens per router tile
+constexpr int kRouterStages = 3;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -56,14 +60,53 @@ inline cudaStream_t S(void* s) { return (cudaStream_t)s; }
 
 }  // namespace
 
+// Optional per-stage timing: CUDA events recorded on the caller's stream around each
+// stage of moe_route / moe_forward, summed by moe_plan_stage_ms.
+struct StageProfiler {
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  struct Rec { int stage; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  int open_stage = -1;
+  cudaEvent_t open_ev = nullptr;
+  cudaEvent_t next() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+  void begin(int stage, cudaStream_t s) {
+    if (!on) return;
+    open_stage = stage;
+    open_ev = next();
+    if (open_ev) cudaEventRecord(open_ev, s);
+  }
+  void end(cudaStream_t s) {
+    if (!on || !open_ev) return;
+    cudaEvent_t b = next();
+    if (!b) return;
+    cudaEventRecord(b, s);
+    recs.push_back({open_stage, open_ev, b});
+    open_ev = nullptr;
+  }
+  ~StageProfiler() {
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
 struct moe_plan_s {
+  StageProfiler prof;
   int T_max, d, E, k, I, Is;
   int num_sms = 148;
   int last_T = 0;
+  int pf_dist = 0, pf_b = 0;  // GEMM L2 prefetch (moe_plan_set_option)
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
-  size_t o_status, o_bias0, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits,
+  size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits,
       o_planes, o_xq, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
   int tokens_per_chunk() const { return kPermThreads; }
   int nchunks(int T) const { return (T + kPermThreads - 1) / kPermThreads; }
@@ -76,7 +119,6 @@ static void carve(moe_plan_s* p) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = up(o + bytes, 1024); return r; };
   p->o_status = take(256);
-  p->o_bias0 = take((size_t)p->E * 4);
   p->o_chunk = take((size_t)p->nchunks(p->T_max) * p->E * 4);
   p->o_counts = take((size_t)p->E * 4);
   p->o_offsets = take((size_t)(p->E + 1) * 4);
@@ -116,6 +158,8 @@ static GemmArgs base_args(const moe_plan_s* p) {
   memset(&a, 0, sizeof(a));
   a.status = p->at<unsigned int>(p->o_status);
   a.dense_rows = -1;
+  a.pf_dist = p->pf_dist;
+  a.pf_b = p->pf_b;
   return a;
 }
 
@@ -266,33 +310,37 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   __nv_bfloat16* planes = p->at<__nv_bfloat16>(p->o_planes);
   float* z = logits_opt ? logits_opt : p->at<float>(p->o_logits);
   if (!aligned(z, 16)) return MOE_ERR_ALIGNMENT;
+  p->prof.begin(MOE_STAGE_ROUTER_SPLIT, s);
   router_split_kernel<<<dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s>>>(W_r, d, E, planes);
-  float* zero_bias = nullptr;
-  if (!bias) {
-    zero_bias = p->at<float>(p->o_bias0);
-    if (cudaMemsetAsync(zero_bias, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
-  }
+  p->prof.end(s);
   CUtensorMap tA, tB;
-  if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, planes, 3ull * d, E, 3ull * d * 2, 64, 256) ||
+  if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, planes, 3ull * d, E, 3ull * d * 2, 64, 128) ||
       !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64, 32))
     return MOE_ERR_CUDA;
-  GemmArgs a = base_args(p);
-  a.dense_rows = T;
-  a.num_groups = 1;
-  a.M_total = E;
-  a.m_tiles = (E + 255) / 256;
-  a.k_tiles = 3 * d / 64;
-  a.kb_wrap = d / 64;
-  a.B_rows = T;
-  a.out0 = z;
-  a.ld_out = E;
-  a.bias = bias ? bias : zero_bias;
-  const int tiles = ((T + kBN - 1) / kBN) * a.m_tiles;
-  if (launch_gemm<KIND_BF16, EPI_LOGITS>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  RouterArgs ra;
+  ra.T = T;
+  ra.d = d;
+  ra.E = E;
+  ra.m_tiles = (E + 127) / 128;
+  ra.bias = bias;
+  ra.z = z;
+  ra.status = p->at<unsigned int>(p->o_status);
+  {
+    using RC = RouterCfg<kRouterBN, kRouterStages>;
+    auto kern = router_kernel<kRouterBN, kRouterStages>;
+    static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RC::SMEM_BYTES);
+    if (attr != cudaSuccess) return MOE_ERR_CUDA;
+    const int tiles = ((T + kRouterBN - 1) / kRouterBN) * ra.m_tiles;
+    p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
+    kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    p->prof.end(s);
+  }
   if (set_smem_attrs() != cudaSuccess) return MOE_ERR_CUDA;
   const int wpb = 8;
+  p->prof.begin(MOE_STAGE_TOPK, s);
   topk_sigmoid_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * E * 4, s>>>(z, T, E, p->k, idx, w);
+  p->prof.end(s);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   p->last_T = T;
   return MOE_OK;
@@ -318,14 +366,18 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   const int A = T * k;
 
   // a4: group assignments by expert
+  p->prof.begin(MOE_STAGE_PERMUTE, s);
   if (run_permute(p, idx, T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  p->prof.end(s);
   // a1: quantise x to MXFP8 and scatter rows into expert order
   uint8_t* xq = p->at<uint8_t>(p->o_xq);
   uint32_t* xs = p->at<uint32_t>(p->o_xs);
   {
     const long long n = (long long)T * (d / 32);
+    p->prof.begin(MOE_STAGE_QUANT, s);
     quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
         (const uint16_t*)x, T, d, k, p->at<int>(p->o_inv), A, xq, xs);
+    p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
   uint8_t* hq = p->at<uint8_t>(p->o_hq);
@@ -352,7 +404,9 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.out0 = hq;
     a.out1 = hs;
     a.ld_out = I;
+    p->prof.begin(MOE_STAGE_GATE_UP, s);
     if (launch_gemm<KIND_MX, EPI_GLU_MX8>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    p->prof.end(s);
   }
   // a7: down grouped GEMM -> O (bf16, expert order)
   {
@@ -374,7 +428,9 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.sfb = hs;
     a.out0 = O;
     a.ld_out = d;
+    p->prof.begin(MOE_STAGE_DOWN, s);
     if (launch_gemm<KIND_MX, EPI_BF16>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    p->prof.end(s);
   }
   // a8: shared expert (bf16)
   float* ys = nullptr;
@@ -396,8 +452,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.out0 = hsh;
     a.ld_out = Is;
     int tiles = ((T + kBN - 1) / kBN) * a.m_tiles;
+    p->prof.begin(MOE_STAGE_SHARED_GATE_UP, s);
     if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
       return MOE_ERR_CUDA;
+    p->prof.end(s);
     CUtensorMap tA2, tB2;
     if (!make_map(&tA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sh->w_dn, Is, d, (uint64_t)Is * 2, 64, 256) ||
         !make_map(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hsh, Is, T, (uint64_t)Is * 2, 64, 32))
@@ -413,11 +471,15 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     b.out0 = ys;
     b.ld_out = d;
     tiles = ((T + kBN - 1) / kBN) * b.m_tiles;
+    p->prof.begin(MOE_STAGE_SHARED_DOWN, s);
     if (launch_gemm<KIND_BF16, EPI_F32>(p, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
       return MOE_ERR_CUDA;
+    p->prof.end(s);
   }
   // a9: weighted combine with the shared output
+  p->prof.begin(MOE_STAGE_COMBINE, s);
   combine_kernel<<<T, 128, k * 8, s>>>(O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
+  p->prof.end(s);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   p->last_T = T;
   return MOE_OK;
@@ -470,6 +532,46 @@ moe_status_t moe_pack_shared_bf16(int d, int Is, const void* wg, const void* wu,
       return MOE_ERR_CUDA;
   }
   if (cudaMemcpyAsync(dst->w_dn, wd, (size_t)d * Is * 2, cudaMemcpyDeviceToDevice, s)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_set_option(moe_plan_t p, int option, int value) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  switch (option) {
+    case MOE_OPT_PREFETCH_DIST:
+      if (value < 0 || value > 64) return MOE_ERR_INVALID_ARG;
+      p->pf_dist = value;
+      return MOE_OK;
+    case MOE_OPT_PREFETCH_B:
+      p->pf_b = value != 0;
+      return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t moe_plan_set_profiling(moe_plan_t p, int enable) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  p->prof.on = enable != 0;
+  p->prof.recs.clear();
+  p->prof.used = 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_stage_ms(moe_plan_t p, float* ms, int* launches, int n) {
+  if (!p || !ms || n < MOE_NUM_STAGES) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    ms[i] = 0.0f;
+    if (launches) launches[i] = 0;
+  }
+  for (const auto& r : p->prof.recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return MOE_ERR_CUDA;
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return MOE_ERR_CUDA;
+    ms[r.stage] += t;
+    if (launches) launches[r.stage] += 1;
+  }
+  p->prof.recs.clear();
+  p->prof.used = 0;
   return MOE_OK;
 }
 

@@ -32,8 +32,7 @@ enum {
   EPI_GLU_MX8 = 0,   // a = silu(gate) * up, requantised to MXFP8 along the channels
   EPI_GLU_BF16 = 1,  // a = silu(gate) * up, stored as bf16
   EPI_BF16 = 2,      // D stored as bf16
-  EPI_F32 = 3,       // D stored as fp32
-  EPI_LOGITS = 4     // D + bias[channel] stored as fp32
+  EPI_F32 = 3        // D stored as fp32
 };
 
 struct GemmArgs {
@@ -52,8 +51,9 @@ struct GemmArgs {
   void* out0;
   void* out1;
   int ld_out;           // elements per output row
-  const float* bias;    // EPI_LOGITS
   unsigned int* status;
+  int pf_dist;          // L2 prefetch distance in k-tiles (0 = off)
+  int pf_b;             // also prefetch the B tiles
 };
 
 template <int KIND, int BN_MAX, int STAGES>
@@ -118,7 +118,7 @@ __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, 
   ti.n_mma = (ti.n_valid + 15) & ~15;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // MXFP8 (E4M3) encoding of v with block scale exponent from the block's amax bits.
 __device__ __forceinline__ int mx_exp_e4m3(uint32_t amax_bits) {
@@ -181,6 +181,28 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
     int stage = 0;
     uint32_t phase = 0;
+    // L2 prefetch cursor, pf_dist k-tiles ahead of the loads along the (tile, k) sequence,
+    // so DRAM latency can be covered by L2 rather than by shared-memory stages.
+    int pf_t = args.pf_dist > 0 ? (int)blockIdx.x : num_tiles, pf_kt = 0;
+    TileInfo pf;
+    if (pf_t < num_tiles) gemm_decode_tile(args, BN_MAX, pf_t, pf);
+    auto prefetch_one = [&]() {
+      if (pf_t >= num_tiles) return;
+      if (lane == 0) {
+        tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
+        if (args.pf_b) {
+          const int kb = pf_kt % args.kb_wrap;
+          const int nb = (pf.n_mma + 31) >> 5;
+          for (int i = 0; i < nb; ++i) tma_prefetch_2d(&tmB, kb * C::BK, pf.row0 + 32 * i);
+        }
+      }
+      if (++pf_kt == args.k_tiles) {
+        pf_kt = 0;
+        pf_t += gridDim.x;
+        if (pf_t < num_tiles) gemm_decode_tile(args, BN_MAX, pf_t, pf);
+      }
+    };
+    for (int i = 0; i < args.pf_dist; ++i) prefetch_one();
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
@@ -223,6 +245,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int i = 0; i < nB; ++i)
             tma_load_2d(smem_u32(sB + i * 4096), &tmB, fb, kb * C::BK, ti.row0 + 32 * i, pol_b);
         }
+        prefetch_one();
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -302,62 +325,111 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
       tc_fence_after();
       const int nchunks = ti.n_mma >> 4;
+      constexpr int CH = BN_MAX / 16;
+      auto release_tmem = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+      };
       if constexpr (EPI == EPI_GLU_MX8 || EPI == EPI_GLU_BF16) {
-        const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
-        for (int c = sub; c < nchunks; c += 2) {
-          uint32_t g[16], u[16];
-          tmem_ld16(lane_base + c * 16, g);
-          tmem_ld16(lane_base + BN_MAX + c * 16, u);
-          tmem_ld_wait();
+        // a = silu(g) * u for this warp's chunks (c = sub + 2 i) straight out of TMEM;
+        // TMEM goes back to the MMA warp before the quantisation and stores.
+        float a[CH / 2][16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = c * 16 + i;
+        for (int i = 0; i < CH / 2; ++i) {
+          const int c = sub + 2 * i;
+          if (c < nchunks) {
+            uint32_t g[16], u[16];
+            tmem_ld16(lane_base + c * 16, g);
+            tmem_ld16(lane_base + BN_MAX + c * 16, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a[i][j] = silu_f(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+          }
+        }
+        release_tmem();
+        const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
+#pragma unroll
+        for (int i = 0; i < CH / 2; ++i) {
+          const int c = sub + 2 * i;
+          if (c >= nchunks) break;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c * 16 + j;
             if (n >= ti.n_valid) break;
-            const float gv = __uint_as_float(g[i]);
-            const float a = silu_f(gv) * __uint_as_float(u[i]);
             const size_t row = (size_t)(ti.row0 + n);
             if constexpr (EPI == EPI_GLU_MX8) {
-              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a) & 0x7FFFFFFFu);
+              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a[i][j]) & 0x7FFFFFFFu);
               const int e = mx_exp_e4m3(amax);
-              const float qv = a * __uint_as_float((uint32_t)(127 - e) << 23);
+              const float qv = a[i][j] * __uint_as_float((uint32_t)(127 - e) << 23);
               const uint32_t code = f32x2_to_e4m3x2(qv, 0.0f) & 0xFFu;
               ((uint8_t*)args.out0)[row * args.ld_out + ch] = (uint8_t)code;
               if (lane == 0)
                 ((uint8_t*)args.out1)[((size_t)ti.mt * args.B_rows + row) * 4 + q] = (uint8_t)(e + 127);
             } else {
-              ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a);
+              ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a[i][j]);
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_BF16) {
+        // round to bf16 pairs while draining TMEM, release it, then store
+        const int h = sub;
+        const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
+        uint32_t v[CH][8];
+        if (half_ok) {
+#pragma unroll
+          for (int c = 0; c < CH; ++c)
+            if (c < nchunks) {
+              uint32_t r[16];
+              tmem_ld16(lane_base + h * BN_MAX + c * 16, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const __nv_bfloat162 p2 =
+                    __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                v[c][j] = *(const uint32_t*)&p2;
+              }
+            }
+        }
+        release_tmem();
+        const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
+        if (half_ok && ch < args.M_total) {
+          uint16_t* out = (uint16_t*)args.out0;
+#pragma unroll
+          for (int c = 0; c < CH; ++c) {
+            if (c >= nchunks) break;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c * 16 + j;
+              if (n >= ti.n_valid) break;
+              out[(size_t)(ti.row0 + n) * args.ld_out + ch] = (uint16_t)(v[c][j >> 1] >> ((j & 1) * 16));
             }
           }
         }
       } else {
+        // fp32 results: store straight from TMEM chunk by chunk, release at the end
         const int h = sub;
         const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
         const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
         if (half_ok) {
           const bool ch_ok = ch < args.M_total;
-          float bias = 0.0f;
-          if constexpr (EPI == EPI_LOGITS) bias = ch_ok ? __ldg(args.bias + ch) : 0.0f;
           for (int c = 0; c < nchunks; ++c) {
             uint32_t v[16];
             tmem_ld16(lane_base + h * BN_MAX + c * 16, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int n = c * 16 + i;
+            for (int j = 0; j < 16; ++j) {
+              const int n = c * 16 + j;
               if (n >= ti.n_valid) break;
               if (!ch_ok) continue;
-              const size_t o = (size_t)(ti.row0 + n) * args.ld_out + ch;
-              const float x = __uint_as_float(v[i]);
-              if constexpr (EPI == EPI_BF16) ((__nv_bfloat16*)args.out0)[o] = __float2bfloat16_rn(x);
-              else ((float*)args.out0)[o] = x + bias;
+              ((float*)args.out0)[(size_t)(ti.row0 + n) * args.ld_out + ch] = __uint_as_float(v[j]);
             }
           }
         }
+        release_tmem();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acc_empty));
       acc_phase ^= 1;
+
     }
   }
 

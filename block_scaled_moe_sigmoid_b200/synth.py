@@ -78,6 +78,9 @@ WORKLOADS = {
     # skewed routing through a Zipf-like logit bias
     "k3_skewed_t32768": Workload("k3_skewed_t32768", 3, 32768, 7168, 896, 16, 3072, 3072,
                                  skew_bias=True, device="cuda"),
+    # Kimi-K3 expert shapes on a 64-expert slice (2.2 GB of weights): a profiling case that
+    # keeps the device footprint to a few GB while the weights still exceed L2
+    "k3_slice_e64_t1024": Workload("k3_slice_e64_t1024", 2, 1024, 7168, 64, 16, 3072, 3072, device="cuda"),
     # token-count sweep (T is given per run)
     "k3_sweep": Workload("k3_sweep", 4, 1, 7168, 896, 16, 3072, 3072, device="cuda",
                          sweep=(1, 16, 256, 2048, 16384)),

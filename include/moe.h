@@ -23,7 +23,7 @@
  *   - Matrices are row-major.  Weights are stored out x in (row = output channel).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL = legacy
  *     default stream); none synchronises the host except moe_plan_check and
- *     moe_debug_read_status.
+ *     moe_plan_stage_ms.
  *   - Errors are returned as moe_status_t; nothing is thrown.  Argument checks happen
  *     before any launch, so an error return leaves outputs untouched.
  *   - Device-side faults (an out-of-range expert id, a pipeline wait that timed out) are
@@ -152,6 +152,35 @@ moe_status_t moe_pack_expert_mxfp4(int d, int I, int e, const float* w_gate, con
  * dst (device buffers of 2*I_s*d and d*I_s bf16). */
 moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const void* w_up,
                                   const void* w_down, const moe_shared_bf16* dst, void* stream);
+
+/* ---- tuning options ----------------------------------------------------------------
+ * MOE_OPT_PREFETCH_DIST: the grouped GEMMs issue L2 prefetches of their weight tiles this
+ *   many K tiles ahead of the shared-memory loads (0..64, 0 = off).
+ * MOE_OPT_PREFETCH_B: non-zero also prefetches the token-row tiles. */
+enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1 };
+moe_status_t moe_plan_set_option(moe_plan_t plan, int option, int value);
+
+/* ---- per-stage timing ---------------------------------------------------------------
+ * With profiling on, every stage of moe_route / moe_forward is bracketed by two CUDA
+ * events recorded on the call's stream (no host synchronisation).  moe_plan_stage_ms
+ * synchronises on them and returns, per stage, the summed elapsed milliseconds and the
+ * number of recorded launches since profiling was enabled or last queried (host arrays of
+ * n >= MOE_NUM_STAGES entries; `launches` may be NULL), then forgets them. */
+enum {
+  MOE_STAGE_ROUTER_SPLIT = 0,    /* W_r -> three bf16 planes */
+  MOE_STAGE_ROUTER_GEMM = 1,     /* logits on the tensor cores */
+  MOE_STAGE_TOPK = 2,            /* sigmoid top-k + renormalise */
+  MOE_STAGE_PERMUTE = 3,         /* histogram, scan, placement (3 kernels) */
+  MOE_STAGE_QUANT = 4,           /* MXFP8 quantise + scatter to expert order */
+  MOE_STAGE_GATE_UP = 5,         /* routed gate/up GEMM + GLU + MXFP8 requant */
+  MOE_STAGE_DOWN = 6,            /* routed down GEMM */
+  MOE_STAGE_SHARED_GATE_UP = 7,  /* shared expert gate/up + GLU */
+  MOE_STAGE_SHARED_DOWN = 8,     /* shared expert down */
+  MOE_STAGE_COMBINE = 9,         /* weighted combine */
+  MOE_NUM_STAGES = 10
+};
+moe_status_t moe_plan_set_profiling(moe_plan_t plan, int enable);
+moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n);
 
 /* ---- introspection (tests) ----------------------------------------------------------
  * Device pointer and size of a workspace buffer after a call, for checking the steps:
