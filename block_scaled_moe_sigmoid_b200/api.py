@@ -37,6 +37,7 @@ SIGNATURES = {
     "moe_debug_buffer": [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_S)],
     "moe_plan_set_profiling": [_P, _I],
     "moe_plan_set_option": [_P, _I, _I],
+    "moe_permute_noalloc": [_P, _I, _I, _I, _P, _P, _P, _P, _P],
     "moe_plan_stage_ms": [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _I],
 }
 
@@ -148,6 +149,21 @@ def moe_permute(plan, idx, E, stream=None):
     inv = torch.empty((T, k), dtype=torch.int32, device=dev)
     _call("moe_permute", plan, _ptr(idx), T, _ptr(counts), _ptr(offsets), _ptr(perm_tok), _ptr(inv),
           _stream(stream))
+    return counts, offsets, perm_tok, inv
+
+
+def moe_permute_noalloc(idx, E, stream=None):
+    """moe_permute for callers that cannot allocate device memory: the library uses its own
+    fixed device scratch array (see include/moe.h for the size limit).  The output
+    tensors here are allocated by torch for convenience."""
+    T, k = idx.shape
+    dev = idx.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm_tok = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty((T, k), dtype=torch.int32, device=dev)
+    _call("moe_permute_noalloc", _ptr(idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm_tok),
+          _ptr(inv), _stream(stream))
     return counts, offsets, perm_tok, inv
 
 

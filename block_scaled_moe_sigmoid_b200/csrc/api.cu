@@ -596,3 +596,63 @@ moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- grouping without allocation
+// Fixed device scratch for moe_permute_noalloc: status word, per-chunk expert counts and
+// the tile table.  Every device that loads this library keeps it until the process exits.
+static constexpr size_t kNoAllocScratchBytes = 256 * 1024;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device (with
+// that device current) and cached.
+static void* noalloc_scratch(moe_status_t* st) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = MOE_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      *st = MOE_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+extern "C" moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                                            int32_t* offsets, int32_t* perm_tok, int32_t* inv,
+                                            void* stream) {
+  if (T < 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (k > E || k > 32 || E > 4096) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !offsets || (T > 0 && (!idx || !perm_tok || !inv))) return MOE_ERR_INVALID_ARG;
+  const int nch = (T + kPermThreads - 1) / kPermThreads;
+  const size_t o_chunk = 256, o_tiles = o_chunk + up((size_t)nch * E * 4, 256);
+  if (o_tiles + (size_t)(E + 1) * 4 > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = S(stream);
+  if (T == 0) {
+    if (cudaMemsetAsync(counts, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  moe_status_t st = MOE_OK;
+  char* scratch = (char*)noalloc_scratch(&st);
+  if (!scratch) return st;
+  if (set_smem_attrs() != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned int* status = (unsigned int*)scratch;
+  int* chunk = (int*)(scratch + o_chunk);
+  int* tiles = (int*)(scratch + o_tiles);
+  // the status word is the only part read before it is written: clear it
+  if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  perm_histogram_kernel<<<nch, 256, E * 4, s>>>(idx, T, k, E, kPermThreads, chunk, status);
+  perm_scan_kernel<<<1, 1024, (2 * E + 32) * 4, s>>>(chunk, nch, E, kBN, counts, offsets, tiles);
+  perm_place_kernel<<<nch, kPermThreads, (kPermThreads / 32) * E * 4, s>>>(idx, T, k, E, kPermThreads,
+                                                                         chunk, perm_tok, inv);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

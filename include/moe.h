@@ -127,6 +127,26 @@ moe_status_t moe_route(moe_plan_t plan, const void* x_bf16, int T, const float* 
 moe_status_t moe_permute(moe_plan_t plan, const int32_t* idx, int T, int32_t* counts,
                          int32_t* offsets, int32_t* perm_tok, int32_t* inv, void* stream);
 
+/* ---- a4 without device allocation ---------------------------------------------------
+ * The same grouping as moe_permute, for callers that cannot call cudaMalloc: code that
+ * runs inside a host application or serving engine which owns the whole device-memory
+ * budget (and may forbid or account every allocation), or a thread that must not take the
+ * allocator's locks or risk the implicit device synchronisation of cudaMalloc/cudaFree.
+ * It needs no plan and no workspace.  The source pages have no counterpart; this is a
+ * deployment aid of this library.
+ * Scratch: a fixed 256 KiB array in the library's device memory, held by every GPU that
+ * loads the library until the process exits.  Calls are rejected with
+ * MOE_ERR_UNSUPPORTED_SHAPE when 256 + ceil(T/256)*E*4 (rounded up to 256) + (E+1)*4
+ * bytes exceed it (e.g. T <= 18432 at E = 896).  All calls share the array, so two calls
+ * whose work overlaps on the GPU (different streams, or different host threads) race.
+ * The first call on a device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture.
+ * Arguments and outputs as moe_permute (device pointers, caller-owned); ids outside
+ * [0, E) are skipped and leave inv = -1 (no status is reported). */
+moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                                 int32_t* offsets, int32_t* perm_tok, int32_t* inv,
+                                 void* stream);
+
 /* ---- a4..a9: the layer ----------------------------------------------------------------
  * y = bf16( shared(x) + sum_j w[t][j] * expert_{idx[t][j]}(x) ), where an expert is
  * down(silu(x Wg^T) * (x Wu^T)) on MXFP8 x and MXFP4 weights, its GLU output requantised
