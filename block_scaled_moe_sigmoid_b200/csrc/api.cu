@@ -54,6 +54,14 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Token-row maps for the grouped GEMM: box heights 32, 64, ... rows (one per tile size).
+bool make_bmaps(BMaps* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+                uint64_t row_bytes, uint32_t box_inner) {
+  for (int i = 0; i < MAX_BOX; ++i)
+    if (!make_map(&m->box[i], dt, base, inner, rows, row_bytes, box_inner, 32u * (i + 1))) return false;
+  return true;
+}
+
 inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 inline size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline cudaStream_t S(void* s) { return (cudaStream_t)s; }
@@ -139,7 +147,7 @@ static void carve(moe_plan_s* p) {
 
 template <int KIND, int EPI>
 static cudaError_t launch_gemm(const moe_plan_s* p, const GemmArgs& a, const CUtensorMap& tA,
-                               const CUtensorMap& tB, int grid, cudaStream_t s) {
+                               const BMaps& tB, int grid, cudaStream_t s) {
   using Cfg = GemmCfg<KIND, kBN, kStages>;
   auto kern = gemm_kernel<KIND, EPI, kBN, kStages>;
   static bool attr_set = false;
@@ -385,9 +393,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   __nv_bfloat16* O = p->at<__nv_bfloat16>(p->o_O);
   // a5/a6: gate/up grouped GEMM, SiLU-GLU and MXFP8 requantisation in the epilogue
   {
-    CUtensorMap tA, tB;
+    CUtensorMap tA;
+    BMaps tB;
     if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, d, (uint64_t)E * 2 * I, d / 2, 128, 256) ||
-        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, d, A, d, 128, 32))
+        !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, d, A, d, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
     a.counts = p->at<int>(p->o_counts);
@@ -410,9 +419,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   }
   // a7: down grouped GEMM -> O (bf16, expert order)
   {
-    CUtensorMap tA, tB;
+    CUtensorMap tA;
+    BMaps tB;
     if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_dn, I, (uint64_t)E * d, I / 2, 128, 256) ||
-        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, A, I, 128, 32))
+        !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, A, I, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
     a.counts = p->at<int>(p->o_counts);
@@ -437,9 +447,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   if (sh) {
     __nv_bfloat16* hsh = p->at<__nv_bfloat16>(p->o_hsh);
     ys = p->at<float>(p->o_ys);
-    CUtensorMap tA, tB;
+    CUtensorMap tA;
+    BMaps tB;
     if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sh->w_gu, d, 2ull * Is, (uint64_t)d * 2, 64, 256) ||
-        !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64, 32))
+        !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
     a.dense_rows = T;
@@ -456,9 +467,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
       return MOE_ERR_CUDA;
     p->prof.end(s);
-    CUtensorMap tA2, tB2;
+    CUtensorMap tA2;
+    BMaps tB2;
     if (!make_map(&tA2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, sh->w_dn, Is, d, (uint64_t)Is * 2, 64, 256) ||
-        !make_map(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hsh, Is, T, (uint64_t)Is * 2, 64, 32))
+        !make_bmaps(&tB2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hsh, Is, T, (uint64_t)Is * 2, 64))
       return MOE_ERR_CUDA;
     GemmArgs b = base_args(p);
     b.dense_rows = T;

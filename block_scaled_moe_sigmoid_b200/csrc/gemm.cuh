@@ -19,9 +19,10 @@
 // covers group-tile t / m_tiles and weight m-tile t % m_tiles, so CTAs running at the
 // same time share the group's B rows through L2.
 //
-// Roles (320 threads): warp 0 loads (TMA for A/B tiles, bulk copy for A scales,
-// cp.async for B scales), warp 1 owns TMEM and one lane issues the MMAs, warps 2..9
-// run the epilogue (lane quarter = warp % 4).
+// Roles (352 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
+// scales), warp 10 loads the token rows (one TMA box, plus cp.async of their scales),
+// warp 1 owns TMEM and one lane issues the MMAs, warps 2..9 run the epilogue (lane
+// quarter = warp % 4).  The two producers fill the same stage independently.
 #pragma once
 #include "ptx.cuh"
 
@@ -71,7 +72,7 @@ struct GemmCfg {
   static constexpr int TMEM_SFA = 2 * BN_MAX;                  // 4 columns per half
   static constexpr int TMEM_SFB = 2 * BN_MAX + 8;              // 4 columns per 128 B rows
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NUM_THREADS = 320;
+  static constexpr int NUM_THREADS = 352;
   static_assert(BN_MAX % 32 == 0 && BN_MAX <= 256, "BN_MAX");
   static_assert(TMEM_SFB + 4 * SFB_ATOMS <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
@@ -132,10 +133,16 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Token-row tensor maps with box heights 32, 64, ..., 32 * MAX_BOX rows.
+constexpr int MAX_BOX = 8;
+struct BMaps {
+  CUtensorMap box[MAX_BOX];
+};
+
 template <int KIND, int EPI, int BN_MAX, int STAGES>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     gemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA,
-                const __grid_constant__ CUtensorMap tmB) {
+                const __grid_constant__ BMaps tmB) {
   using C = GemmCfg<KIND, BN_MAX, STAGES>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 33 : 1);
+      mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 34 : 2);  // 2 producers (+32 cp.async)
       mbar_init(smem_u32(empty_bar + s), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
@@ -162,7 +169,6 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -176,26 +182,19 @@ __global__ void __launch_bounds__(320, 1)
   const int num_tiles = gemm_num_tiles(args, BN_MAX);
 
   if (warp == 0) {
-    // ------------------------------------------------------------- producer
+    // ------------------------------------------------------------- producer: weights
+    // One TMA box of 256 weight rows x one K tile, plus (KIND_MX) a 1 KB bulk copy of
+    // the matching scale-factor atoms.
     const uint64_t pol_a = policy_evict_first();  // weights stream through once
-    const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
     int stage = 0;
     uint32_t phase = 0;
-    // L2 prefetch cursor, pf_dist k-tiles ahead of the loads along the (tile, k) sequence,
-    // so DRAM latency can be covered by L2 rather than by shared-memory stages.
+    // L2 prefetch cursor, pf_dist k-tiles ahead of the loads along the (tile, k) sequence.
     int pf_t = args.pf_dist > 0 ? (int)blockIdx.x : num_tiles, pf_kt = 0;
     TileInfo pf;
     if (pf_t < num_tiles) gemm_decode_tile(args, BN_MAX, pf_t, pf);
     auto prefetch_one = [&]() {
       if (pf_t >= num_tiles) return;
-      if (lane == 0) {
-        tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
-        if (args.pf_b) {
-          const int kb = pf_kt % args.kb_wrap;
-          const int nb = (pf.n_mma + 31) >> 5;
-          for (int i = 0; i < nb; ++i) tma_prefetch_2d(&tmB, kb * C::BK, pf.row0 + 32 * i);
-        }
-      }
+      if (lane == 0) tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
       if (++pf_kt == args.k_tiles) {
         pf_kt = 0;
         pf_t += gridDim.x;
@@ -203,24 +202,57 @@ __global__ void __launch_bounds__(320, 1)
       }
     };
     for (int i = 0; i < args.pf_dist; ++i) prefetch_one();
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
       const int a_row = ti.grp * args.M_total + ti.mt * C::BM;
+      for (int kt = 0; kt < args.k_tiles; ++kt) {
+        if (lane == 0) {
+          ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
+          if (ok) {
+            uint8_t* sA = smem + stage * C::STAGE_BYTES;
+            const uint32_t fb = smem_u32(full_bar + stage);
+            mbar_arrive_expect_tx(fb, C::A_TX + C::SFA_BYTES);
+            tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
+            if constexpr (KIND == KIND_MX) {
+              const uint8_t* sfa_src =
+                  args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
+              asm volatile(
+                  "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::
+                      "r"(smem_u32(sA + C::A_BYTES + C::B_BYTES)),
+                  "l"(sfa_src), "r"(fb)
+                  : "memory");
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        prefetch_one();
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------- producer: token rows
+    // One TMA box of the tile's rows (box height 32 * nB, nB = ceil(n_mma / 32)) and
+    // (KIND_MX) the rows' scale words by cp.async into the scale-factor atom layout:
+    // row n -> atom n/128, byte (n%32)*16 + ((n%128)/32)*4.
+    const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      TileInfo ti;
+      gemm_decode_tile(args, BN_MAX, t, ti);
       const int nB = (ti.n_mma + 31) >> 5;
-      bool ok = true;
       for (int kt = 0; kt < args.k_tiles; ++kt) {
         if (lane == 0) ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
-        uint8_t* sA = smem + stage * C::STAGE_BYTES;
-        uint8_t* sB = sA + C::A_BYTES;
-        uint8_t* sSFA = sB + C::B_BYTES;
-        uint8_t* sSFB = sSFA + C::SFA_BYTES;
+        uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
         const uint32_t fb = smem_u32(full_bar + stage);
         if constexpr (KIND == KIND_MX) {
-          // B scales: one 32-bit word (4 K-blocks) per token row, into the MMA's
-          // scale-factor atom layout: row n -> atom n/128, byte (n%32)*16 + ((n%128)/32)*4.
+          uint8_t* sSFB = sB + C::B_BYTES + C::SFA_BYTES;
           const uint32_t* src = args.sfb + (size_t)kt * args.B_rows + ti.row0;
           for (int n = lane; n < ti.n_valid; n += 32) {
             const uint32_t off = (n >> 7) * 512 + (n & 31) * 16 + ((n & 127) >> 5) * 4;
@@ -229,27 +261,12 @@ __global__ void __launch_bounds__(320, 1)
           cp_async_mbar_arrive_noinc(fb);
         }
         if (lane == 0) {
-          const uint32_t tx = C::A_TX + nB * 4096 + C::SFA_BYTES;
-          mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
-          if constexpr (KIND == KIND_MX) {
-            const uint8_t* sfa_src =
-                args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
-            asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::
-                    "r"(smem_u32(sSFA)),
-                "l"(sfa_src), "r"(fb)
-                : "memory");
-          }
-          const int kb = kt % args.kb_wrap;
-          for (int i = 0; i < nB; ++i)
-            tma_load_2d(smem_u32(sB + i * 4096), &tmB, fb, kb * C::BK, ti.row0 + 32 * i, pol_b);
+          mbar_arrive_expect_tx(fb, nB * 4096);
+          tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
         }
-        prefetch_one();
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
