@@ -19,10 +19,11 @@
 // covers group-tile t / m_tiles and weight m-tile t % m_tiles, so CTAs running at the
 // same time share the group's B rows through L2.
 //
-// Roles (352 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
+// Roles (384 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
 // scales), warp 10 loads the token rows (one TMA box, plus cp.async of their scales),
-// warp 1 owns TMEM and one lane issues the MMAs, warps 2..9 run the epilogue (lane
-// quarter = warp % 4).  The two producers fill the same stage independently.
+// warp 11 copies each stage's scale factors into TMEM (KIND_MX), warp 1 owns TMEM and one
+// lane issues the MMAs, warps 2..9 run the epilogue (lane quarter = warp % 4).  The two
+// producers fill the same stage independently.
 #pragma once
 #include "ptx.cuh"
 
@@ -69,12 +70,14 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int A_TX = KIND == KIND_MX ? BM * BK / 2 : BM * BK * 2;  // global bytes
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
-  static constexpr int TMEM_SFA = 2 * BN_MAX;                  // 4 columns per half
-  static constexpr int TMEM_SFB = 2 * BN_MAX + 8;              // 4 columns per 128 B rows
+  // scale factors in TMEM, one 16-column buffer per pipeline stage:
+  //   A: 4 columns per 128-row half (+0, +4), B: 4 columns per 128 token rows (+8, +12)
+  static constexpr int TMEM_SF = 2 * BN_MAX;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int NUM_THREADS = 352;
+  static constexpr int NUM_THREADS = 384;
   static_assert(BN_MAX % 32 == 0 && BN_MAX <= 256, "BN_MAX");
-  static_assert(TMEM_SFB + 4 * SFB_ATOMS <= TMEM_COLS, "TMEM budget");
+  static_assert(SFB_ATOMS <= 2, "scale buffer holds two B atoms");
+  static_assert(TMEM_SF + 16 * STAGES <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -140,7 +143,7 @@ struct BMaps {
 };
 
 template <int KIND, int EPI, int BN_MAX, int STAGES>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     gemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ BMaps tmB) {
   using C = GemmCfg<KIND, BN_MAX, STAGES>;
@@ -149,10 +152,12 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t* ctrl = smem + STAGES * C::STAGE_BYTES;
   uint64_t* full_bar = (uint64_t*)ctrl;
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* acc_full = empty_bar + STAGES;
+  uint64_t* sf_ready = empty_bar + STAGES;       // scale factors of the stage are in TMEM
+  uint64_t* acc_full = sf_ready + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain_bar = acc_empty + 1;
-  uint32_t* tmem_holder = (uint32_t*)(drain_bar + 1);
+  uint64_t* drain_sf = drain_bar + 1;
+  uint32_t* tmem_holder = (uint32_t*)(drain_sf + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -162,10 +167,12 @@ __global__ void __launch_bounds__(352, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 34 : 2);  // 2 producers (+32 cp.async)
       mbar_init(smem_u32(empty_bar + s), 1);
+      mbar_init(smem_u32(sf_ready + s), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(acc_empty), 8);
     mbar_init(smem_u32(drain_bar), 1);
+    mbar_init(smem_u32(drain_sf), 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
@@ -268,6 +275,39 @@ __global__ void __launch_bounds__(352, 1)
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------- scale factors -> TMEM
+    // tcgen05.cp of each stage's scale atoms into that stage's TMEM buffer, off the MMA
+    // thread's instruction stream.  A buffer is rewritten only after the stage was
+    // refilled, i.e. after the MMAs that read it committed.
+    if (KIND == KIND_MX && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        TileInfo ti;
+        gemm_decode_tile(args, BN_MAX, t, ti);
+        const bool h1 = ti.mt * C::BM + 128 < args.M_total;
+        const int atoms = (ti.n_mma + 127) >> 7;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
+          const uint32_t sSFB = sSFA + C::SFA_BYTES;
+          const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
+          tc_cp_32x128b_warpx4(tsf, smem_desc(sSFA, 16, 128, 0));
+          if (h1) tc_cp_32x128b_warpx4(tsf + 4, smem_desc(sSFA + 512, 16, 128, 0));
+          for (int a = 0; a < atoms; ++a)
+            tc_cp_32x128b_warpx4(tsf + 8 + 4 * a, smem_desc(sSFB + 512 * a, 16, 128, 0));
+          tc_commit(smem_u32(sf_ready + stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      tc_commit(smem_u32(drain_sf));
+      mbar_wait(smem_u32(drain_sf), 0, args.status, abort_flag);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -283,19 +323,12 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         for (int kt = 0; kt < args.k_tiles; ++kt) {
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
+          if (ok && KIND == KIND_MX) ok = mbar_wait(smem_u32(sf_ready + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
-          if constexpr (KIND == KIND_MX) {
-            const uint32_t sSFA = sB + C::B_BYTES;
-            const uint32_t sSFB = sSFA + C::SFA_BYTES;
-            tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFA, smem_desc(sSFA, 16, 128, 0));
-            if (h1) tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFA + 4, smem_desc(sSFA + 512, 16, 128, 0));
-            const int atoms = (ti.n_mma + 127) >> 7;
-            for (int a = 0; a < atoms; ++a)
-              tc_cp_32x128b_warpx4(tmem_base + C::TMEM_SFB + 4 * a, smem_desc(sSFB + 512 * a, 16, 128, 0));
-          }
+          const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t bdesc = smem_desc(sB + 32 * j, 16, 1024, 2);
@@ -307,8 +340,8 @@ __global__ void __launch_bounds__(352, 1)
               const uint32_t d_tmem = tmem_base + h * BN_MAX;
               if constexpr (KIND == KIND_MX) {
                 const uint32_t idesc = idesc_mx_e2m1_e4m3(128, ti.n_mma, j, j);
-                const uint32_t sfa = (tmem_base + C::TMEM_SFA + 4 * h) | ((uint32_t)j << 30);
-                const uint32_t sfb = (tmem_base + C::TMEM_SFB) | ((uint32_t)j << 30);
+                const uint32_t sfa = (tsf + 4 * h) | ((uint32_t)j << 30);
+                const uint32_t sfb = (tsf + 8) | ((uint32_t)j << 30);
                 mma_mxf8f6f4(d_tmem, adesc, bdesc, idesc, sfa, sfb, acc);
               } else {
                 mma_bf16(d_tmem, adesc, bdesc, idesc_bf16(128, ti.n_mma), acc);
