@@ -136,9 +136,11 @@ static void carve(moe_plan_s* p) {
   p->o_logits = take((size_t)p->T_max * p->E * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
   p->o_xq = take(A * p->d);
-  p->o_xs = take((size_t)(p->d / 128) * A * 4);
+  // token-side scale blocks, tile-major: at most A / kBN + E group-tiles
+  const size_t max_tiles = A / kBN + p->E + 1;
+  p->o_xs = take(max_tiles * (p->d / 128) * SF_TILE_BYTES);
   p->o_hq = take(A * p->I);
-  p->o_hs = take((size_t)(p->I / 128) * A * 4);
+  p->o_hs = take(max_tiles * (p->I / 128) * SF_TILE_BYTES);
   p->o_O = take(A * p->d * 2);
   p->o_hsh = take((size_t)p->T_max * (p->Is ? p->Is : 1) * 2);
   p->o_ys = take((size_t)p->T_max * p->d * 4);
@@ -379,23 +381,25 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   p->prof.end(s);
   // a1: quantise x to MXFP8 and scatter rows into expert order
   uint8_t* xq = p->at<uint8_t>(p->o_xq);
-  uint32_t* xs = p->at<uint32_t>(p->o_xs);
+  uint8_t* xs = p->at<uint8_t>(p->o_xs);
   {
     const long long n = (long long)T * (d / 32);
     p->prof.begin(MOE_STAGE_QUANT, s);
     quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-        (const uint16_t*)x, T, d, k, p->at<int>(p->o_inv), A, xq, xs);
+        (const uint16_t*)x, T, d, k, idx, p->at<int>(p->o_inv), p->at<int>(p->o_counts),
+        p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), A, xq, xs);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
   uint8_t* hq = p->at<uint8_t>(p->o_hq);
-  uint32_t* hs = p->at<uint32_t>(p->o_hs);
+  uint8_t* hs = p->at<uint8_t>(p->o_hs);
   __nv_bfloat16* O = p->at<__nv_bfloat16>(p->o_O);
   // a5/a6: gate/up grouped GEMM, SiLU-GLU and MXFP8 requantisation in the epilogue
   {
     CUtensorMap tA;
     BMaps tB;
-    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, d, (uint64_t)E * 2 * I, d / 2, 128, 256) ||
+    // tile-major weights: 128-element rows of 64 B, one 256-row box per (expert, m-tile, k-tile)
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, 128, (uint64_t)E * 2 * I * (d / 128), 64, 128, 256) ||
         !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, d, A, d, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
@@ -421,7 +425,8 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   {
     CUtensorMap tA;
     BMaps tB;
-    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_dn, I, (uint64_t)E * d, I / 2, 128, 256) ||
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_dn, 128,
+                  (uint64_t)E * ((d + 255) / 256) * 256 * (I / 128), 64, 128, 256) ||
         !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, A, I, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
@@ -502,7 +507,7 @@ moe_status_t moe_expert_bytes(int d, int I, int E, size_t* w_gu, size_t* s_gu, s
   if (d % 128 || I % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
   *w_gu = (size_t)E * 2 * I * (d / 2);
   *s_gu = (size_t)E * (2 * I / 256) * (d / 128) * 1024;
-  *w_dn = (size_t)E * d * (I / 2);
+  *w_dn = (size_t)E * ((d + 255) / 256) * 256 * (I / 2);
   *s_dn = (size_t)E * ((d + 255) / 256) * (I / 128) * 1024;
   return MOE_OK;
 }
@@ -516,13 +521,14 @@ moe_status_t moe_pack_expert_mxfp4(int d, int I, int e, const float* wg, const f
   if (!aligned(wg, 16) || !aligned(wu, 16) || !aligned(wd, 16)) return MOE_ERR_ALIGNMENT;
   cudaStream_t s = S(stream);
   const size_t gu_w = (size_t)2 * I * (d / 2), gu_s = (size_t)(2 * I / 256) * (d / 128) * 1024;
-  const size_t dn_w = (size_t)d * (I / 2), dn_s = (size_t)((d + 255) / 256) * (I / 128) * 1024;
+  const size_t dn_w = (size_t)((d + 255) / 256) * 256 * (I / 2), dn_s = (size_t)((d + 255) / 256) * (I / 128) * 1024;
   uint8_t* wgu = (uint8_t*)dst->w_gu + (size_t)e * gu_w;
   uint8_t* sgu = (uint8_t*)dst->s_gu + (size_t)e * gu_s;
   uint8_t* wdn = (uint8_t*)dst->w_dn + (size_t)e * dn_w;
   uint8_t* sdn = (uint8_t*)dst->s_dn + (size_t)e * dn_s;
-  // the down scales' last tile may have an unused half: keep it defined
+  // the down weights' last 256-row tile may have an unused half: keep it defined
   if (cudaMemsetAsync(sdn, 0, dn_s, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (d % 256 && cudaMemsetAsync(wdn, 0, dn_w, s) != cudaSuccess) return MOE_ERR_CUDA;
   long long n = 2ll * I * (d / 32);
   pack_mxfp4_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(wg, wu, I, d, 1, wgu, sgu);
   n = (long long)d * (I / 32);
@@ -594,9 +600,9 @@ moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes
   size_t off, n;
   switch (which) {
     case 0: off = p->o_xq; n = A * p->d; break;
-    case 1: off = p->o_xs; n = (p->d / 128) * A * 4; break;
+    case 1: off = p->o_xs; n = (A / kBN + p->E + 1) * (p->d / 128) * SF_TILE_BYTES; break;
     case 2: off = p->o_hq; n = A * p->I; break;
-    case 3: off = p->o_hs; n = (p->I / 128) * A * 4; break;
+    case 3: off = p->o_hs; n = (A / kBN + p->E + 1) * (p->I / 128) * SF_TILE_BYTES; break;
     case 4: off = p->o_O; n = A * p->d * 2; break;
     case 5: off = p->o_ys; n = T * p->d * 4; break;
     case 6: off = p->o_logits; n = T * p->E * 4; break;

@@ -10,7 +10,9 @@
 // Kinds:
 //   KIND_MX:   tcgen05.mma kind::mxf8f6f4.block_scale, A = E2M1 (MXFP4 weights, loaded by
 //              TMA with the 16U4_ALIGN16B unpacking type), B = E4M3 (MXFP8 activations),
-//              one E8M0 scale per 32 K-elements on both sides, fp32 accumulation.
+//              one E8M0 scale per 32 K-elements on both sides, fp32 accumulation.  The
+//              weights are stored tile-major, [group][m-tile][k-tile][256 rows][64 B], so
+//              each stage's weight tile is one contiguous 16 KB block in HBM.
 //   KIND_BF16: tcgen05.mma kind::f16 with bf16 A and B, fp32 accumulation.
 //
 // Groups: rows of B are grouped (one group per expert, contiguous rows
@@ -20,12 +22,13 @@
 // same time share the group's B rows through L2.
 //
 // Roles (384 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
-// scales), warp 10 loads the token rows (one TMA box, plus cp.async of their scales),
+// scales), warp 10 loads the token rows (one TMA box, plus a bulk copy of their scales),
 // warp 11 copies each stage's scale factors into TMEM (KIND_MX), warp 1 owns TMEM and one
 // lane issues the MMAs, warps 2..9 run the epilogue (lane quarter = warp % 4).  The two
 // producers fill the same stage independently.
 #pragma once
 #include "ptx.cuh"
+#include "tiling.cuh"
 
 namespace moe {
 
@@ -49,7 +52,7 @@ struct GemmArgs {
   int kb_wrap;      // B's K-tile coordinate is taken modulo kb_wrap
   int B_rows;       // rows of the B tensor
   const uint8_t* sfa;   // KIND_MX: A scales, [G][m_tiles][k_tiles][2 halves][512 B atom]
-  const uint32_t* sfb;  // KIND_MX: B scales, words [k_tiles][B_rows], byte j = K-block 4kt+j
+  const uint8_t* sfb;   // KIND_MX: B scales, tile-major [group-tiles][k_tiles][1 KB] (tiling.cuh)
   void* out0;
   void* out1;
   int ld_out;           // elements per output row
@@ -83,7 +86,7 @@ struct GemmCfg {
 };
 
 struct TileInfo {
-  int grp, mt, row0, n_valid, n_mma;
+  int grp, gt, mt, row0, n_valid, n_mma;  // gt: group-tile index
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const GemmArgs& a, int bn_max) {
@@ -114,9 +117,9 @@ __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, 
     Me = __ldg(a.counts + grp);
     base = __ldg(a.offsets + grp);
   }
-  int n_per = (Me + ntiles - 1) / ntiles;
-  n_per = (n_per + 15) & ~15;
+  const int n_per = tile_rows_per(Me, ntiles);
   ti.grp = grp;
+  ti.gt = gt;
   ti.row0 = base + nt * n_per;
   ti.n_valid = min(n_per, Me - nt * n_per);
   ti.n_mma = (ti.n_valid + 15) & ~15;
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 34 : 2);  // 2 producers (+32 cp.async)
+      mbar_init(smem_u32(full_bar + s), 2);  // one arrival per producer warp
       mbar_init(smem_u32(empty_bar + s), 1);
       mbar_init(smem_u32(sf_ready + s), 1);
     }
@@ -201,7 +204,12 @@ __global__ void __launch_bounds__(384, 1)
     if (pf_t < num_tiles) gemm_decode_tile(args, BN_MAX, pf_t, pf);
     auto prefetch_one = [&]() {
       if (pf_t >= num_tiles) return;
-      if (lane == 0) tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
+      if (lane == 0) {
+        if constexpr (KIND == KIND_MX)
+          tma_prefetch_2d(&tmA, 0, ((pf.grp * args.m_tiles + pf.mt) * args.k_tiles + pf_kt) * C::BM);
+        else
+          tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
+      }
       if (++pf_kt == args.k_tiles) {
         pf_kt = 0;
         pf_t += gridDim.x;
@@ -221,7 +229,10 @@ __global__ void __launch_bounds__(384, 1)
             uint8_t* sA = smem + stage * C::STAGE_BYTES;
             const uint32_t fb = smem_u32(full_bar + stage);
             mbar_arrive_expect_tx(fb, C::A_TX + C::SFA_BYTES);
-            tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
+            if constexpr (KIND == KIND_MX)   // tile-major weights: one contiguous 16 KB block
+              tma_load_2d(smem_u32(sA), &tmA, fb, 0, ((ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * C::BM, pol_a);
+            else
+              tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
             if constexpr (KIND == KIND_MX) {
               const uint8_t* sfa_src =
                   args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
@@ -242,8 +253,7 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 10) {
     // ------------------------------------------------------------- producer: token rows
     // One TMA box of the tile's rows (box height 32 * nB, nB = ceil(n_mma / 32)) and
-    // (KIND_MX) the rows' scale words by cp.async into the scale-factor atom layout:
-    // row n -> atom n/128, byte (n%32)*16 + ((n%128)/32)*4.
+    // (KIND_MX) one bulk copy of the tile's scale atoms for this K tile.
     const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
     int stage = 0;
     uint32_t phase = 0;
@@ -258,18 +268,18 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
         const uint32_t fb = smem_u32(full_bar + stage);
-        if constexpr (KIND == KIND_MX) {
-          uint8_t* sSFB = sB + C::B_BYTES + C::SFA_BYTES;
-          const uint32_t* src = args.sfb + (size_t)kt * args.B_rows + ti.row0;
-          for (int n = lane; n < ti.n_valid; n += 32) {
-            const uint32_t off = (n >> 7) * 512 + (n & 31) * 16 + ((n & 127) >> 5) * 4;
-            cp_async_4(smem_u32(sSFB + off), src + n);
-          }
-          cp_async_mbar_arrive_noinc(fb);
-        }
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, nB * 4096);
+          const int sfb_bytes = KIND == KIND_MX ? ((ti.n_mma + 127) >> 7) * 512 : 0;
+          mbar_arrive_expect_tx(fb, nB * 4096 + sfb_bytes);
           tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
+          if constexpr (KIND == KIND_MX) {
+            const uint8_t* src = args.sfb + ((size_t)ti.gt * args.k_tiles + kt) * SF_TILE_BYTES;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+                    "r"(smem_u32(sB + C::B_BYTES + C::SFA_BYTES)),
+                "l"(src), "r"(sfb_bytes), "r"(fb)
+                : "memory");
+          }
         }
         __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -414,8 +424,9 @@ __global__ void __launch_bounds__(384, 1)
               const float qv = a[i][j] * __uint_as_float((uint32_t)(127 - e) << 23);
               const uint32_t code = f32x2_to_e4m3x2(qv, 0.0f) & 0xFFu;
               ((uint8_t*)args.out0)[row * args.ld_out + ch] = (uint8_t)code;
-              if (lane == 0)
-                ((uint8_t*)args.out1)[((size_t)ti.mt * args.B_rows + row) * 4 + q] = (uint8_t)(e + 127);
+              if (lane == 0)   // scale byte for the down GEMM: K tile mt, block q, tile-major
+                ((uint8_t*)args.out1)[((size_t)ti.gt * args.m_tiles + ti.mt) * SF_TILE_BYTES +
+                                      sf_atom_offset(n) + q] = (uint8_t)(e + 127);
             } else {
               ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a[i][j]);
             }

@@ -3,6 +3,7 @@
 // weighted combine, and the setup-time weight packers (MXFP4 experts, bf16 router planes).
 #pragma once
 #include "ptx.cuh"
+#include "tiling.cuh"
 
 namespace moe {
 
@@ -77,12 +78,14 @@ __global__ void quant_mxfp8_kernel(const uint16_t* __restrict__ x, int rows, int
   sc[r * nb + b] = (uint8_t)s;
 }
 
-// Quantise token rows and write each to its k positions in expert order:
-// xq[inv[t][j]][:] and the scale words xs[(block/4)][inv[t][j]] (byte block%4).
-// Requires cols % 128 == 0 so four consecutive threads share a row and one word.
+// Quantise token rows and write each to its k positions in expert order: the elements to
+// xq[inv[t][j]][:], the scales tile-major (tiling.cuh) for the gate/up GEMM.
+// Requires cols % 128 == 0 so four consecutive threads share a row and one scale word.
 __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int cols, int k,
-                                     const int* __restrict__ inv, int A_rows,
-                                     uint8_t* __restrict__ xq, uint32_t* __restrict__ xs) {
+                                     const int* __restrict__ idx, const int* __restrict__ inv,
+                                     const int* __restrict__ counts, const int* __restrict__ offsets,
+                                     const int* __restrict__ tile_prefix, int A_rows,
+                                     uint8_t* __restrict__ xq, uint8_t* __restrict__ xs) {
   const int nb = cols >> 5;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const bool active = gid < (long long)T * nb;
@@ -105,13 +108,18 @@ __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int 
   const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
   const uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
   const uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
+  const int k_tiles = cols >> 7;
   for (int j = 0; j < k; ++j) {
     const int p = __ldg(inv + t * k + j);
     if (p < 0 || p >= A_rows) continue;
     uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
     dst[0] = o0;
     dst[1] = o1;
-    if ((l & 3) == 0) xs[(size_t)(b >> 2) * A_rows + p] = word;
+    if ((l & 3) == 0) {
+      int gt, n;
+      row_tile(counts, offsets, tile_prefix, __ldg(idx + t * k + j), p, gt, n);
+      *(uint32_t*)(xs + ((size_t)gt * k_tiles + (b >> 2)) * SF_TILE_BYTES + sf_atom_offset(n)) = word;
+    }
   }
 }
 
@@ -334,8 +342,9 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ O, const float*
 }
 
 // ---------------------------------------------------------------- weight packing (setup)
-// fp32 rows [R][K] -> E2M1 codes (2 per byte, element 2j in the low nibble) at packed row
-// dst_row(r), and E8M0 scales into the MMA scale-factor atom layout
+// fp32 rows [R][K] -> E2M1 codes (2 per byte, element 2j in the low nibble) for packed row
+// dst_row(r) in the tile-major code layout [m-tile][K/128][256 rows][64 B], and E8M0
+// scales into the MMA scale-factor atom layout
 // [m_tiles][K/128][2][512]: row rr of a 256-row tile, K-block kb ->
 //   ((mt * (K/128) + kb/4) * 2 + half) * 512 + (rr%32)*16 + ((rr%128)/32)*4 + kb%4.
 // interleave != 0: rows of two sources (gate, up) go to packed rows
@@ -373,7 +382,9 @@ __global__ void pack_mxfp4_kernel(const float* __restrict__ src0, const float* _
     wds[i] = acc;
   }
   const int pr = interleave ? 256 * (r >> 7) + 128 * which + (r & 127) : r;
-  *(uint4*)(wdst + (size_t)pr * (K / 2) + b * 16) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  // tile-major codes: [m-tile][k-tile][256 rows][64 B]; block b is 16 B of its row's 64 B
+  const size_t wo = ((size_t)((pr >> 8) * (K >> 7) + (b >> 2)) * 256 + (pr & 255)) * 64 + (b & 3) * 16;
+  *(uint4*)(wdst + wo) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
   const int mt = pr >> 8, half = (pr >> 7) & 1, rr = pr & 127;
   const size_t so = ((size_t)(mt * (K >> 7) + (b >> 2)) * 2 + half) * 512 + (rr & 31) * 16 +
                     (rr >> 5) * 4 + (b & 3);

@@ -56,12 +56,14 @@ typedef enum { MOE_ACT_SILU_GLU = 0 } moe_act_t;
 typedef enum { MOE_BIAS_LOGIT = 0 } moe_bias_mode_t;
 
 /* Packed MXFP4 expert weights (device pointers, all 256-byte aligned).
- *   w_gu: E2M1 codes of gate and up, [E][2I][d/2] bytes, element 2j of a row in the low
- *         nibble of byte j.  Rows are channel blocks of 128 interleaved as
- *         gate[0:128], up[0:128], gate[128:256], up[128:256], ...
- *   s_gu: E8M0 scales (one per 32 elements along d) in the tensor-core scale-factor
- *         tiling [E][2I/256][d/128][2][512] (see moe_pack_expert_mxfp4).
- *   w_dn: E2M1 codes of down, [E][d][I/2] bytes.
+ *   Rows of gate and up are channel blocks of 128 interleaved as gate[0:128], up[0:128],
+ *   gate[128:256], up[128:256], ... (2I packed rows); down has d rows (output channels).
+ *   w_gu: E2M1 codes, tile-major [E][2I/256][d/128][256 rows][64 B]: 128 consecutive input
+ *         elements of a packed row per 64 bytes, element 2j in the low nibble of byte j.
+ *   s_gu: E8M0 scales (one per 32 input elements) in the tensor-core scale-factor tiling
+ *         [E][2I/256][d/128][2][512]: packed row r of a 256-row tile, 32-block b of the
+ *         K tile -> half r/128, byte (r%32)*16 + ((r%128)/32)*4 + b.
+ *   w_dn: E2M1 codes of down, [E][ceil(d/256)][I/128][256][64 B] (rows past d are zero).
  *   s_dn: E8M0 scales of down, [E][ceil(d/256)][I/128][2][512].
  * Sizes come from moe_expert_bytes; contents from moe_pack_expert_mxfp4. */
 typedef struct {
@@ -205,9 +207,12 @@ moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n)
 /* ---- introspection (tests) ----------------------------------------------------------
  * Device pointer and size of a workspace buffer after a call, for checking the steps:
  *   0 xq  E4M3 [T*k][d] activations in expert order
- *   1 xs  u32 scale words [d/128][T*k] (byte j = 32-block 4m+j of a row)
+ *   1 xs  scales of xq, tile-major: for group-tile g (tiles of <= 160 rows per expert,
+ *         ceil(count/160) tiles of round16(ceil(count/tiles)) rows each, numbered in
+ *         expert order) and 128-column K tile kt, 1 KB at (g*(d/128) + kt)*1024; row n of
+ *         the tile, 32-block j of the K tile at (n/128)*512 + (n%32)*16 + ((n%128)/32)*4 + j
  *   2 hq  E4M3 [T*k][I] GLU output in expert order
- *   3 hs  u32 scale words [I/128][T*k]
+ *   3 hs  scales of hq, same tile-major layout with I/128 K tiles
  *   4 O   bf16 [T*k][d] expert outputs in expert order
  *   5 ys  fp32 [T][d] shared expert output
  *   6 logits fp32 [T][E]

@@ -10,15 +10,22 @@ from oracle import layer, mx, router
 
 def unpack_expert_codes(ex, e, d, I):
     """Packed w_gu / s_gu / w_dn / s_dn of expert e -> plain (codes, scales) per matrix,
-    following the layout documented in include/moe.h."""
+    following the tile-major layouts documented in include/moe.h."""
+    mt_dn = (d + 255) // 256
     gu_w = 2 * I * d // 2
     gu_s = (2 * I // 256) * (d // 128) * 1024
-    dn_w = d * I // 2
-    dn_s = ((d + 255) // 256) * (I // 128) * 1024
-    wgu = ex.w_gu[e * gu_w:(e + 1) * gu_w].cpu().numpy().reshape(2 * I, d // 2)
+    dn_w = mt_dn * 256 * I // 2
+    dn_s = mt_dn * (I // 128) * 1024
+    wgu = ex.w_gu[e * gu_w:(e + 1) * gu_w].cpu().numpy()
     sgu = ex.s_gu[e * gu_s:(e + 1) * gu_s].cpu().numpy()
-    wdn = ex.w_dn[e * dn_w:(e + 1) * dn_w].cpu().numpy().reshape(d, I // 2)
+    wdn = ex.w_dn[e * dn_w:(e + 1) * dn_w].cpu().numpy()
     sdn = ex.s_dn[e * dn_s:(e + 1) * dn_s].cpu().numpy()
+
+    def codes(buf, rows, K):
+        # [m-tile][k-tile][256][64 B] -> [rows][K/2]
+        mt = -(-rows // 256)
+        t = buf.reshape(mt, K // 128, 256, 64).transpose(0, 2, 1, 3).reshape(mt * 256, K // 2)
+        return t[:rows]
 
     def scales(buf, rows, K):
         pr = np.arange(rows)[:, None]
@@ -27,7 +34,7 @@ def unpack_expert_codes(ex, e, d, I):
         off = ((mt * (K // 128) + (b >> 2)) * 2 + half) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (b & 3)
         return buf[off]
 
-    codes_gu = mx.unpack_e2m1(wgu)
+    codes_gu = mx.unpack_e2m1(codes(wgu, 2 * I, d))
     sc_gu = scales(sgu, 2 * I, d)
     # rows are interleaved in 128-row blocks: gate[0:128], up[0:128], gate[128:256], ...
     c = np.arange(I)
@@ -36,8 +43,30 @@ def unpack_expert_codes(ex, e, d, I):
     return {
         "gate": (codes_gu[g_rows], sc_gu[g_rows]),
         "up": (codes_gu[u_rows], sc_gu[u_rows]),
-        "down": (mx.unpack_e2m1(wdn), scales(sdn, d, I)),
+        "down": (mx.unpack_e2m1(codes(wdn, d, I)), scales(sdn, d, I)),
     }
+
+
+def decode_tile_major_scales(buf, counts, k_tiles, bn=160):
+    """Token-side scale bytes [A][k_tiles*4] from the tile-major layout documented in
+    include/moe.h (debug buffers 1 and 3), using the expert row counts."""
+    buf = np.asarray(buf, dtype=np.uint8)
+    rows = []
+    gt = 0
+    for c in counts:
+        c = int(c)
+        if c == 0:
+            continue
+        ntiles = -(-c // bn)
+        n_per = -(-c // ntiles)
+        n_per = (n_per + 15) // 16 * 16
+        for r in range(c):
+            nt, n = divmod(r, n_per)
+            off = (n >> 7) * 512 + (n & 31) * 16 + ((n & 127) >> 5) * 4
+            base = (gt + nt) * k_tiles * 1024 + off
+            rows.append(np.concatenate([buf[base + kt * 1024: base + kt * 1024 + 4] for kt in range(k_tiles)]))
+        gt += ntiles
+    return np.stack(rows) if rows else np.zeros((0, 4 * k_tiles), np.uint8)
 
 
 class Case:

@@ -11,7 +11,7 @@ import torch
 from block_scaled_moe_sigmoid_b200 import api, synth
 from oracle import layer, mx, permute as operm, router
 
-from .gpu_helpers import Case, layer_stats, unpack_expert_codes
+from .gpu_helpers import Case, decode_tile_major_scales, layer_stats, unpack_expert_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -146,19 +146,21 @@ def _stage_checks(case, idx, w):
     """Intermediates in expert order against the oracle on the same routing."""
     wl, T = case.wl, case.T
     A = T * wl.k
-    _, offs, perm_tok, inv = operm.permute(idx, wl.E)
+    counts, offs, perm_tok, inv = operm.permute(idx, wl.E)
     x = case.x_np()
     xq_ref, xs_ref = mx.quantize_mx(x, "e4m3")
     xq = case.plan.debug_tensor(0, torch.uint8, (A, wl.d)).cpu().numpy()
-    xs = case.plan.debug_tensor(1, torch.int32, (wl.d // 128, A)).cpu().numpy().view(np.uint8)
-    xs = xs.reshape(wl.d // 128, A, 4).transpose(1, 0, 2).reshape(A, wl.d // 32)
+    ptr, nbytes = api.moe_debug_buffer(case.plan.handle, 1)
+    xs = decode_tile_major_scales(case.plan.debug_tensor(1, torch.uint8, (nbytes,)).cpu().numpy(),
+                                  counts, wl.d // 128)
     assert np.array_equal(xq, xq_ref[perm_tok])
     assert np.array_equal(xs, xs_ref[perm_tok])
     # GLU output (MXFP8): decoded values agree up to one E4M3 step where fp32 and fp64
     # land on different sides of a rounding boundary
     hq = case.plan.debug_tensor(2, torch.uint8, (A, wl.I)).cpu().numpy()
-    hs = case.plan.debug_tensor(3, torch.int32, (wl.I // 128, A)).cpu().numpy().view(np.uint8)
-    hs = hs.reshape(wl.I // 128, A, 4).transpose(1, 0, 2).reshape(A, wl.I // 32)
+    ptr, nbytes = api.moe_debug_buffer(case.plan.handle, 3)
+    hs = decode_tile_major_scales(case.plan.debug_tensor(3, torch.uint8, (nbytes,)).cpu().numpy(),
+                                  counts, wl.I // 128)
     H = mx.dequantize_mx(hq, hs, "e4m3")
     X = mx.dequantize_mx(xq_ref, xs_ref, "e4m3")
     worst, mism = 0.0, 0
