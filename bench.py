@@ -27,6 +27,12 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s at K3 shape (T=8192); % FP4 tensor peak, decode % HBM BW"
 UNIT = "tokens/s"
 
+# DRAM bytes (read + write) of one launch of the routed gate/up GEMM on the T=8192
+# workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` of this
+# kernel version (profiles/dram_gemm_k3_prefill_t8192.md).  None whenever the kernel
+# has changed since that capture.
+GATE_UP_TRAFFIC_BYTES = {8192: 24714007552 + 412475648}
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -268,7 +274,9 @@ def run_ours(args, rank, world, local_rank):
     achieved = flops / (gu_ms / gu_n / 1e3) / 1e12 if gu_n else None
     roofline = {"kernel": "gemm_kernel<KIND_MX, EPI_GLU_MX8> (routed gate/up + SiLU-GLU + MXFP8 requant)",
                 "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak if achieved else None, "traffic": None,
+                "frac": achieved / peak if achieved else None,
+                "traffic": (GATE_UP_TRAFFIC_BYTES.get(T) if args.workload == "k3_prefill_t8192" else None),
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "peak_note": f"FP8-rate tensor pipe = 2 x {peak_src} sustained bf16 GEMM "
                              f"(kind::mxf8f6f4 issues at the FP8 rate)",
                 "ms_per_launch": gu_ms / gu_n if gu_n else None,
