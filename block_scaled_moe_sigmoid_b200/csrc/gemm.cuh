@@ -291,6 +291,8 @@ __global__ void __launch_bounds__(384, 1)
     // thread's instruction stream.  A buffer is rewritten only after the stage was
     // refilled, i.e. after the MMAs that read it committed.
     if (KIND == KIND_MX && lane == 0) {
+      // no-swizzle descriptor of stage 0's A scale atoms (32 rows x 16 B, 128 B per 8 rows)
+      const uint64_t sf_desc0 = smem_desc(smem_u32(smem) + C::A_BYTES + C::B_BYTES, 16, 128, 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -303,13 +305,13 @@ __global__ void __launch_bounds__(384, 1)
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
-          const uint32_t sSFB = sSFA + C::SFA_BYTES;
+          const uint64_t sfa_desc = sf_desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t sfb_desc = sfa_desc + (uint64_t)(C::SFA_BYTES >> 4);
           const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
-          tc_cp_32x128b_warpx4(tsf, smem_desc(sSFA, 16, 128, 0));
-          if (h1) tc_cp_32x128b_warpx4(tsf + 4, smem_desc(sSFA + 512, 16, 128, 0));
-          for (int a = 0; a < atoms; ++a)
-            tc_cp_32x128b_warpx4(tsf + 8 + 4 * a, smem_desc(sSFB + 512 * a, 16, 128, 0));
+          tc_cp_32x128b_warpx4(tsf, sfa_desc);
+          if (h1) tc_cp_32x128b_warpx4(tsf + 4, sfa_desc + (uint64_t)(512 >> 4));
+          tc_cp_32x128b_warpx4(tsf + 8, sfb_desc);
+          if (atoms > 1) tc_cp_32x128b_warpx4(tsf + 12, sfb_desc + (uint64_t)(512 >> 4));
           tc_commit(smem_u32(sf_ready + stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -321,6 +323,8 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      // 128-byte-swizzled K-major descriptor of stage 0's A tile; other tiles are offsets
+      const uint64_t desc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -328,6 +332,13 @@ __global__ void __launch_bounds__(384, 1)
         TileInfo ti;
         gemm_decode_tile(args, BN_MAX, t, ti);
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
+        // Everything the MMAs of a stage need except the stage offset is fixed per tile:
+        // the issue loop below only adds constants (the tcgen05.mma issue rate is set by
+        // how fast this one thread can form its operands).
+        uint32_t idesc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          idesc[j] = KIND == KIND_MX ? idesc_mx_e2m1_e4m3(128, ti.n_mma, j, j) : idesc_bf16(128, ti.n_mma);
         ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -336,26 +347,23 @@ __global__ void __launch_bounds__(384, 1)
           if (ok && KIND == KIND_MX) ok = mbar_wait(smem_u32(sf_ready + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
+          const uint64_t a_desc = desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t b_desc = a_desc + (uint64_t)(C::A_BYTES >> 4);
           const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
+          const uint32_t acc0 = kt > 0 ? 1u : 0u;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint64_t bdesc = smem_desc(sB + 32 * j, 16, 1024, 2);
-            const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               if (h == 1 && !h1) continue;
-              const uint64_t adesc = smem_desc(sA + h * 16384 + 32 * j, 16, 1024, 2);
-              const uint32_t d_tmem = tmem_base + h * BN_MAX;
-              if constexpr (KIND == KIND_MX) {
-                const uint32_t idesc = idesc_mx_e2m1_e4m3(128, ti.n_mma, j, j);
-                const uint32_t sfa = (tsf + 4 * h) | ((uint32_t)j << 30);
-                const uint32_t sfb = (tsf + 8) | ((uint32_t)j << 30);
-                mma_mxf8f6f4(d_tmem, adesc, bdesc, idesc, sfa, sfb, acc);
-              } else {
-                mma_bf16(d_tmem, adesc, bdesc, idesc_bf16(128, ti.n_mma), acc);
-              }
+              const uint64_t adesc = a_desc + (uint64_t)((h * 16384 + 32 * j) >> 4);
+              const uint64_t bdesc = b_desc + (uint64_t)((32 * j) >> 4);
+              const uint32_t acc = j > 0 ? 1u : acc0;
+              if constexpr (KIND == KIND_MX)
+                mma_mxf8f6f4(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], (tsf + 4 * h) | ((uint32_t)j << 30),
+                             (tsf + 8) | ((uint32_t)j << 30), acc);
+              else
+                mma_bf16(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], acc);
             }
           }
           tc_commit(smem_u32(empty_bar + stage));

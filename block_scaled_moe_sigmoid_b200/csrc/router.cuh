@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t phase = 0;
       uint32_t g = 0;  // chain counter across tiles: buffer g & 1, phase (g >> 1) & 1
       bool ok = true;
+      const uint64_t desc0 = smem_desc(smem_u32(smem), 16, 1024, 2);  // stage 0, plane 0
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int row0 = (t / args.m_tiles) * RBN;
         const int n_mma = (min(RBN, args.T - row0) + 15) & ~15;
@@ -126,15 +127,15 @@ __global__ void __launch_bounds__(320, 1)
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
+          const uint64_t a_desc = desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t b_desc = a_desc + (uint64_t)(C::A_BYTES >> 4);
           const uint32_t d_tmem = tmem_base + b * RBN;
 #pragma unroll
           for (int p = 0; p < 3; ++p)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_bf16(d_tmem, smem_desc(sA + p * C::A_PLANE + 32 * j, 16, 1024, 2),
-                       smem_desc(sB + 32 * j, 16, 1024, 2), idesc, (p | j) ? 1u : 0u);
+              mma_bf16(d_tmem, a_desc + (uint64_t)((p * C::A_PLANE + 32 * j) >> 4), b_desc + (uint64_t)((32 * j) >> 4),
+                       idesc, (p | j) ? 1u : 0u);
           tc_commit(smem_u32(empty_bar + stage));
           tc_commit(smem_u32(pfull + b));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
