@@ -88,25 +88,25 @@ def decode_e4m3(codes):
 
 
 def _round_to_format(q, pos_values, max_mag):
-    """RNE of q onto the positive value list, saturating; returns codes (R1, R2).
+    """RNE of q onto the positive value list, saturating; returns (codes, sign) (R1, R2).
 
     pos_values[i] is the value of code i (sign bit clear), increasing in i, so the
     mantissa LSB of code i is i & 1 and "ties to even" means the even index wins.
+    Magnitudes at or above the largest value land on it (saturation).  Works through the
+    array in chunks of 2^20 elements to stay in cache.
     """
     q = np.asarray(q, dtype=np.float64)
-    a = np.abs(q)
-    sat = a >= max_mag
-    a_c = np.minimum(a, max_mag)
-    lo = np.searchsorted(pos_values, a_c, side="right") - 1      # value[lo] <= a
-    lo = np.clip(lo, 0, len(pos_values) - 1)
-    hi = np.minimum(lo + 1, len(pos_values) - 1)
-    d_lo = a_c - pos_values[lo]
-    d_hi = pos_values[hi] - a_c
-    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi != lo) & (hi % 2 == 0))
-    idx = np.where(pick_hi, hi, lo)
-    idx = np.where(sat, len(pos_values) - 1, idx)
-    sign = np.signbit(q)
-    return idx, sign
+    flat = q.reshape(-1)
+    idx = np.empty(flat.shape, dtype=np.int64)
+    top = len(pos_values) - 1
+    for s0 in range(0, flat.size, 1 << 20):
+        a = np.minimum(np.abs(flat[s0:s0 + (1 << 20)]), max_mag)
+        lo = np.searchsorted(pos_values, a, side="right") - 1      # value[lo] <= a
+        hi = np.minimum(lo + 1, top)
+        d_lo = a - pos_values[lo]
+        d_hi = pos_values[hi] - a
+        idx[s0:s0 + a.size] = np.where((d_hi < d_lo) | ((d_hi == d_lo) & ((hi & 1) == 0)), hi, lo)
+    return idx.reshape(q.shape), np.signbit(q)
 
 
 def block_scale_exponent(amax, emax):
