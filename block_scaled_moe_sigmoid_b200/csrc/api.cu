@@ -413,6 +413,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.kb_wrap = a.k_tiles;
     a.B_rows = A;
     a.sfa = (const uint8_t*)ex->s_gu;
+    a.a_ptr = (const uint8_t*)ex->w_gu;
     a.sfb = xs;
     a.out0 = hq;
     a.out1 = hs;
@@ -440,6 +441,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.kb_wrap = a.k_tiles;
     a.B_rows = A;
     a.sfa = (const uint8_t*)ex->s_dn;
+    a.a_ptr = (const uint8_t*)ex->w_dn;
     a.sfb = hs;
     a.out0 = O;
     a.ld_out = d;

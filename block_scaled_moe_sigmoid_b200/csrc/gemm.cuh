@@ -57,8 +57,9 @@ struct GemmArgs {
   void* out1;
   int ld_out;           // elements per output row
   unsigned int* status;
-  int pf_dist;          // L2 prefetch distance in k-tiles (0 = off)
-  int pf_b;             // also prefetch the B tiles
+  int pf_dist;          // L2 prefetch distance in k-tiles (0 = off), KIND_MX weights
+  int pf_b;             // reserved
+  const uint8_t* a_ptr; // KIND_MX: packed weights (base of the tile-major code array)
 };
 
 template <int KIND, int BN_MAX, int STAGES>
@@ -156,7 +157,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* full_bar = (uint64_t*)ctrl;
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* sf_ready = empty_bar + STAGES;       // scale factors of the stage are in TMEM
-  uint64_t* acc_full = sf_ready + STAGES;
+  uint64_t* sf_full = sf_ready + STAGES;         // scale blocks of the stage are in smem
+  uint64_t* acc_full = sf_full + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain_bar = acc_empty + 1;
   uint64_t* drain_sf = drain_bar + 1;
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(full_bar + s), 2);  // one arrival per producer warp
       mbar_init(smem_u32(empty_bar + s), 1);
       mbar_init(smem_u32(sf_ready + s), 1);
+      mbar_init(smem_u32(sf_full + s), 2);   // weight-scale and token-scale copies
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(acc_empty), 8);
@@ -204,11 +207,12 @@ __global__ void __launch_bounds__(384, 1)
     if (pf_t < num_tiles) gemm_decode_tile(args, BN_MAX, pf_t, pf);
     auto prefetch_one = [&]() {
       if (pf_t >= num_tiles) return;
-      if (lane == 0) {
-        if constexpr (KIND == KIND_MX)
-          tma_prefetch_2d(&tmA, 0, ((pf.grp * args.m_tiles + pf.mt) * args.k_tiles + pf_kt) * C::BM);
-        else
-          tma_prefetch_2d(&tmA, pf_kt * C::BK, pf.grp * args.M_total + pf.mt * C::BM);
+      if constexpr (KIND == KIND_MX) {
+        // the 16 KB weight tile is contiguous: 128 lines of 128 B, 4 per lane
+        const uint8_t* tile = args.a_ptr + (((size_t)pf.grp * args.m_tiles + pf.mt) * args.k_tiles + pf_kt) * (C::BM * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(tile + (i * 32 + lane) * 128));
       }
       if (++pf_kt == args.k_tiles) {
         pf_kt = 0;
@@ -228,18 +232,20 @@ __global__ void __launch_bounds__(384, 1)
           if (ok) {
             uint8_t* sA = smem + stage * C::STAGE_BYTES;
             const uint32_t fb = smem_u32(full_bar + stage);
-            mbar_arrive_expect_tx(fb, C::A_TX + C::SFA_BYTES);
+            mbar_arrive_expect_tx(fb, C::A_TX);
             if constexpr (KIND == KIND_MX)   // tile-major weights: one contiguous 16 KB block
               tma_load_2d(smem_u32(sA), &tmA, fb, 0, ((ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * C::BM, pol_a);
             else
               tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
             if constexpr (KIND == KIND_MX) {
+              const uint32_t sb = smem_u32(sf_full + stage);
+              mbar_arrive_expect_tx(sb, C::SFA_BYTES);
               const uint8_t* sfa_src =
                   args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
               asm volatile(
                   "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::
                       "r"(smem_u32(sA + C::A_BYTES + C::B_BYTES)),
-                  "l"(sfa_src), "r"(fb)
+                  "l"(sfa_src), "r"(sb)
                   : "memory");
             }
           }
@@ -269,15 +275,17 @@ __global__ void __launch_bounds__(384, 1)
         uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
         const uint32_t fb = smem_u32(full_bar + stage);
         if (lane == 0) {
-          const int sfb_bytes = KIND == KIND_MX ? ((ti.n_mma + 127) >> 7) * 512 : 0;
-          mbar_arrive_expect_tx(fb, nB * 4096 + sfb_bytes);
+          mbar_arrive_expect_tx(fb, nB * 4096);
           tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
           if constexpr (KIND == KIND_MX) {
+            const int sfb_bytes = ((ti.n_mma + 127) >> 7) * 512;
+            const uint32_t sb = smem_u32(sf_full + stage);
+            mbar_arrive_expect_tx(sb, sfb_bytes);
             const uint8_t* src = args.sfb + ((size_t)ti.gt * args.k_tiles + kt) * SF_TILE_BYTES;
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
                     "r"(smem_u32(sB + C::B_BYTES + C::SFA_BYTES)),
-                "l"(src), "r"(sfb_bytes), "r"(fb)
+                "l"(src), "r"(sfb_bytes), "r"(sb)
                 : "memory");
           }
         }
@@ -288,8 +296,9 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 11) {
     // ------------------------------------------------------------- scale factors -> TMEM
     // tcgen05.cp of each stage's scale atoms into that stage's TMEM buffer, off the MMA
-    // thread's instruction stream.  A buffer is rewritten only after the stage was
-    // refilled, i.e. after the MMAs that read it committed.
+    // thread's instruction stream, as soon as the small scale blocks land (their own
+    // barrier, ahead of the large tiles).  A buffer is rewritten only after the stage was
+    // released for refilling, i.e. after the MMAs that read it committed.
     if (KIND == KIND_MX && lane == 0) {
       // no-swizzle descriptor of stage 0's A scale atoms (32 rows x 16 B, 128 B per 8 rows)
       const uint64_t sf_desc0 = smem_desc(smem_u32(smem) + C::A_BYTES + C::B_BYTES, 16, 128, 0);
@@ -302,7 +311,7 @@ __global__ void __launch_bounds__(384, 1)
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
         const int atoms = (ti.n_mma + 127) >> 7;
         for (int kt = 0; kt < args.k_tiles; ++kt) {
-          ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
+          ok = mbar_wait(smem_u32(sf_full + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint64_t sfa_desc = sf_desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);

@@ -176,9 +176,9 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
                                   const void* w_down, const moe_shared_bf16* dst, void* stream);
 
 /* ---- tuning options ----------------------------------------------------------------
- * MOE_OPT_PREFETCH_DIST: the grouped GEMMs issue L2 prefetches of their weight tiles this
- *   many K tiles ahead of the shared-memory loads (0..64, 0 = off).
- * MOE_OPT_PREFETCH_B: non-zero also prefetches the token-row tiles. */
+ * MOE_OPT_PREFETCH_DIST: the routed grouped GEMMs prefetch their weight tiles into L2
+ *   this many K tiles ahead of the shared-memory loads (0..64, 0 = off).
+ * MOE_OPT_PREFETCH_B: accepted and ignored (reserved). */
 enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1 };
 moe_status_t moe_plan_set_option(moe_plan_t plan, int option, int value);
 
