@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--T", type=int, default=None, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 160],
+                    help="grouped-GEMM token rows per tile (0 = the library's per-call choice)")
     return ap.parse_args()
 
 
@@ -122,7 +124,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
@@ -183,6 +185,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     x, W_r, bias, plan, ex, sh = setup(wl, T, "cuda")
+    api.moe_plan_set_option(plan.handle, api.MOE_OPT_TILE_N, args.tile_n)
     idx = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
     w = torch.empty((T, wl.k), dtype=torch.float32, device=dev)
     y = torch.empty((T, wl.d), dtype=torch.bfloat16, device=dev)
@@ -260,29 +263,50 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": y.numel() * y.element_size()}
 
     # ---- roofline of the dominant kernel (routed gate/up GEMM)
+    # Its bound is the slower of two terms: the block-scaled MMAs at the tensor pipe's rate
+    # for MXFP4 x MXFP8 operands (kind::mxf8f6f4 issues at the FP8 rate, twice bf16), and
+    # the algorithmic HBM bytes (the touched experts' codes and scales, the MXFP8 token rows
+    # read once, the MXFP8 GLU output written once) at the measured copy bandwidth.
     peaks = {}
     pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(pk_path):
         peaks = json.load(open(pk_path))
+    if peaks.get("bf16_tflops_sustained"):
+        bf16, peak_src = peaks["bf16_tflops_sustained"], "measured"
+    else:
+        bf16, peak_src = 1400.0, "fallback"
+    hbm, hbm_src = (peaks["hbm_gbs"], "measured") if peaks.get("hbm_gbs") else (6650.0, "fallback")
+    touched = int(torch.unique(idx).numel())
     gu_ms, gu_n = stages["gate_up_glu"]
+    t_launch = gu_ms / gu_n / 1e3 if gu_n else None
     A = T * wl.k
     flops = 2.0 * A * wl.d * (2 * wl.I)
-    if peaks.get("bf16_tflops_sustained"):
-        peak, peak_src = 2.0 * peaks["bf16_tflops_sustained"], "measured"
+    gu_bytes = (touched * 2 * wl.I * wl.d * 17 / 32          # E2M1 codes + E8M0 scales
+                + A * wl.d * 33 / 32 + A * wl.I * 33 / 32)     # MXFP8 rows in, GLU rows out
+    tc_peak = 2.0 * bf16
+    tensor_bound = flops / tc_peak / 1e12 >= gu_bytes / hbm / 1e9
+    if tensor_bound:
+        achieved = flops / t_launch / 1e12 if t_launch else None
+        peak, unit = tc_peak, "TFLOP/s"
     else:
-        peak, peak_src = 2.0 * 1400.0, "fallback"
-    achieved = flops / (gu_ms / gu_n / 1e3) / 1e12 if gu_n else None
+        achieved = gu_bytes / t_launch / 1e9 if t_launch else None
+        peak, unit = hbm, "GB/s"
+    traffic = GATE_UP_TRAFFIC_BYTES.get(T) if args.workload == "k3_prefill_t8192" else None
     roofline = {"kernel": "gemm_kernel<KIND_MX, EPI_GLU_MX8> (routed gate/up + SiLU-GLU + MXFP8 requant)",
-                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak if achieved else None,
-                "traffic": (GATE_UP_TRAFFIC_BYTES.get(T) if args.workload == "k3_prefill_t8192" else None),
+                "bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak if achieved else None, "traffic": traffic,
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                "peak_note": f"FP8-rate tensor pipe = 2 x {peak_src} sustained bf16 GEMM "
-                             f"(kind::mxf8f6f4 issues at the FP8 rate)",
+                "peak_note": (f"tensor: FP8-rate pipe = 2 x {peak_src} sustained bf16 GEMM "
+                              f"(kind::mxf8f6f4 issues at the FP8 rate); hbm: {hbm_src} copy bandwidth"),
                 "ms_per_launch": gu_ms / gu_n if gu_n else None,
-                "flops_per_launch": flops}
-    hbm = peaks.get("hbm_gbs", 6650.0)
-    w_bytes = wl.E * 3 * wl.d * wl.I * 17 / 32
+                "flops_per_launch": flops, "algorithmic_bytes_per_launch": gu_bytes,
+                "touched_experts": touched,
+                "tflops_per_launch": flops / t_launch / 1e12 if t_launch else None,
+                "frac_of_nominal_fp4_rate": (flops / t_launch / 1e12 / (4.0 * bf16)) if t_launch else None,
+                "fp4_note": "FP4-rate MMAs (kind::mxf4) need both operands in E2M1; MXFP8 "
+                            "activations run at the FP8 rate, so the FP4 figure is context"}
+    w_bytes = (touched * 3 * wl.d * wl.I * 17 / 32 + 3 * wl.d * wl.I_shared * 2
+               + wl.d * wl.E * 4)
     stage_ms = {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()}
 
     out = None
@@ -296,11 +320,14 @@ def run_ours(args, rank, world, local_rank):
             "config": {"workload": args.workload, "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I,
                        "I_shared": wl.I_shared, "seed": wl.seed, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2: every step streams "
-                             f"{w_bytes / 1e9:.1f} GB of expert weights"},
+                             f"{w_bytes / 1e9:.1f} GB of weights ({touched} touched experts)"},
             "roofline": roofline,
-            "hbm_view": {"weight_bytes_per_step": w_bytes,
+            "gemm_tile_rows": api.moe_plan_get_option(plan.handle, api.MOE_OPT_TILE_N),
+            "hbm_view": {"weight_bytes_per_step": w_bytes, "touched_experts": touched,
                          "achieved_gbs": w_bytes / (ms / args.steps / 1e3) / 1e9,
-                         "peak_gbs": hbm},
+                         "peak_gbs": hbm, "frac": w_bytes / (ms / args.steps / 1e3) / 1e9 / hbm,
+                         "note": "touched experts' MXFP4 weights + bf16 shared expert + fp32 "
+                                 "router matrix per step, over the whole step's time"},
             "stage_ms_per_launch": stage_ms,
             "clocks": clk, "e2e": e2e, "gpu_launches": launches,
         }

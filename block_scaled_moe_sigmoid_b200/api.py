@@ -37,6 +37,7 @@ SIGNATURES = {
     "moe_debug_buffer": [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_S)],
     "moe_plan_set_profiling": [_P, _I],
     "moe_plan_set_option": [_P, _I, _I],
+    "moe_plan_get_option": [_P, _I, ctypes.POINTER(_I)],
     "moe_permute_noalloc": [_P, _I, _I, _I, _P, _P, _P, _P, _P],
     "moe_plan_stage_ms": [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _I],
 }
@@ -202,11 +203,17 @@ def moe_debug_buffer(plan, which):
     return p.value, n.value
 
 
-MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B = 0, 1
+MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B, MOE_OPT_TILE_N = 0, 1, 2
 
 
 def moe_plan_set_option(plan, option, value):
     _call("moe_plan_set_option", plan, option, int(value))
+
+
+def moe_plan_get_option(plan, option):
+    v = ctypes.c_int()
+    _call("moe_plan_get_option", plan, option, ctypes.byref(v))
+    return v.value
 
 
 def moe_plan_set_profiling(plan, enable=True):

@@ -15,8 +15,14 @@ using namespace moe;
 
 namespace {
 
-constexpr int kBN = 160;      // tokens per GEMM tile (MMA N <= 160)
-constexpr int kStages = 4;    // smem pipeline depth of every GEMM
+// Two GEMM tile configurations, chosen per call from the tokens per expert:
+//   large: up to 160 token rows per tile (MMA N <= 160), 4-stage smem ring (54 KB stages);
+//   small: up to 32 token rows per tile, 5-stage ring (38 KB stages).  With a few tokens
+//   per expert the weight stream is the whole cost and the fifth stage keeps another
+//   16 KB weight tile per SM in flight.
+constexpr int kBN = 160, kStages = 4;
+constexpr int kBNSmall = 32, kStagesSmall = 5;
+constexpr int kBNMin = kBNSmall;   // workspace sizing: the most tiles either configuration forms
 constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
 constexpr int kRouterStages = 3;
@@ -111,6 +117,13 @@ struct moe_plan_s {
   int num_sms = 148;
   int last_T = 0;
   int pf_dist = 0, pf_b = 0;  // GEMM L2 prefetch (moe_plan_set_option)
+  int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
+  int last_bn = 0;            // token rows per tile in the last moe_forward
+  // token rows per GEMM tile for a call with T tokens
+  int tile_rows(int T) const {
+    if (tile_n_opt) return tile_n_opt;
+    return (long long)T * k <= 8ll * E ? kBNSmall : kBN;   // <= 8 tokens per expert on average
+  }
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
@@ -136,8 +149,8 @@ static void carve(moe_plan_s* p) {
   p->o_logits = take((size_t)p->T_max * p->E * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
   p->o_xq = take(A * p->d);
-  // token-side scale blocks, tile-major: at most A / kBN + E group-tiles
-  const size_t max_tiles = A / kBN + p->E + 1;
+  // token-side scale blocks, tile-major: at most A / bn + E group-tiles
+  const size_t max_tiles = A / kBNMin + p->E + 1;
   p->o_xs = take(max_tiles * (p->d / 128) * SF_TILE_BYTES);
   p->o_hq = take(A * p->I);
   p->o_hs = take(max_tiles * (p->I / 128) * SF_TILE_BYTES);
@@ -147,11 +160,11 @@ static void carve(moe_plan_s* p) {
   p->total = o;
 }
 
-template <int KIND, int EPI>
-static cudaError_t launch_gemm(const moe_plan_s* p, const GemmArgs& a, const CUtensorMap& tA,
-                               const BMaps& tB, int grid, cudaStream_t s) {
-  using Cfg = GemmCfg<KIND, kBN, kStages>;
-  auto kern = gemm_kernel<KIND, EPI, kBN, kStages>;
+template <int KIND, int EPI, int BN, int STAGES>
+static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
+                                   cudaStream_t s) {
+  using Cfg = GemmCfg<KIND, BN, STAGES>;
+  auto kern = gemm_kernel<KIND, EPI, BN, STAGES>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
@@ -161,6 +174,13 @@ static cudaError_t launch_gemm(const moe_plan_s* p, const GemmArgs& a, const CUt
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s>>>(a, tA, tB);
   return cudaGetLastError();
+}
+
+template <int KIND, int EPI>
+static cudaError_t launch_gemm(int bn, const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
+                               cudaStream_t s) {
+  if (bn == kBNSmall) return launch_gemm_cfg<KIND, EPI, kBNSmall, kStagesSmall>(a, tA, tB, grid, s);
+  return launch_gemm_cfg<KIND, EPI, kBN, kStages>(a, tA, tB, grid, s);
 }
 
 static GemmArgs base_args(const moe_plan_s* p) {
@@ -184,13 +204,13 @@ static cudaError_t set_smem_attrs() {
 }
 
 // histogram -> scan -> placement into the plan workspace
-static cudaError_t run_permute(moe_plan_s* p, const int32_t* idx, int T, cudaStream_t s) {
+static cudaError_t run_permute(moe_plan_s* p, const int32_t* idx, int T, int bn, cudaStream_t s) {
   if (set_smem_attrs() != cudaSuccess) return cudaErrorInvalidValue;
   const int nch = p->nchunks(T);
   int* chunk = p->at<int>(p->o_chunk);
   perm_histogram_kernel<<<nch, 256, p->E * 4, s>>>(idx, T, p->k, p->E, p->tokens_per_chunk(), chunk,
                                                    p->at<unsigned int>(p->o_status));
-  perm_scan_kernel<<<1, 1024, (2 * p->E + 32) * 4, s>>>(chunk, nch, p->E, kBN, p->at<int>(p->o_counts),
+  perm_scan_kernel<<<1, 1024, (2 * p->E + 32) * 4, s>>>(chunk, nch, p->E, bn, p->at<int>(p->o_counts),
                                                          p->at<int>(p->o_offsets), p->at<int>(p->o_tiles));
   perm_place_kernel<<<nch, kPermThreads, (kPermThreads / 32) * p->E * 4, s>>>(
       idx, T, p->k, p->E, p->tokens_per_chunk(), chunk, p->at<int>(p->o_perm), p->at<int>(p->o_inv));
@@ -295,7 +315,7 @@ moe_status_t moe_permute(moe_plan_t p, const int32_t* idx, int T, int32_t* count
     if (cudaMemsetAsync(offsets, 0, (p->E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  if (run_permute(p, idx, T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (run_permute(p, idx, T, p->tile_rows(T), s) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t A = (size_t)T * p->k;
   if (cudaMemcpyAsync(counts, p->ws + p->o_counts, p->E * 4, cudaMemcpyDeviceToDevice, s) ||
       cudaMemcpyAsync(offsets, p->ws + p->o_offsets, (p->E + 1) * 4, cudaMemcpyDeviceToDevice, s) ||
@@ -374,10 +394,11 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   cudaStream_t s = S(stream);
   const int d = p->d, E = p->E, k = p->k, I = p->I, Is = p->Is;
   const int A = T * k;
+  const int bn = p->tile_rows(T);
 
   // a4: group assignments by expert
   p->prof.begin(MOE_STAGE_PERMUTE, s);
-  if (run_permute(p, idx, T, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (run_permute(p, idx, T, bn, s) != cudaSuccess) return MOE_ERR_CUDA;
   p->prof.end(s);
   // a1: quantise x to MXFP8 and scatter rows into expert order
   uint8_t* xq = p->at<uint8_t>(p->o_xq);
@@ -419,7 +440,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.out1 = hs;
     a.ld_out = I;
     p->prof.begin(MOE_STAGE_GATE_UP, s);
-    if (launch_gemm<KIND_MX, EPI_GLU_MX8>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_gemm<KIND_MX, EPI_GLU_MX8>(bn, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
   // a7: down grouped GEMM -> O (bf16, expert order)
@@ -446,7 +467,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.out0 = O;
     a.ld_out = d;
     p->prof.begin(MOE_STAGE_DOWN, s);
-    if (launch_gemm<KIND_MX, EPI_BF16>(p, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_gemm<KIND_MX, EPI_BF16>(bn, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
   // a8: shared expert (bf16)
@@ -469,9 +490,9 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.B_rows = T;
     a.out0 = hsh;
     a.ld_out = Is;
-    int tiles = ((T + kBN - 1) / kBN) * a.m_tiles;
+    int tiles = ((T + bn - 1) / bn) * a.m_tiles;
     p->prof.begin(MOE_STAGE_SHARED_GATE_UP, s);
-    if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(p, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
+    if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
       return MOE_ERR_CUDA;
     p->prof.end(s);
     CUtensorMap tA2;
@@ -489,18 +510,20 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     b.B_rows = T;
     b.out0 = ys;
     b.ld_out = d;
-    tiles = ((T + kBN - 1) / kBN) * b.m_tiles;
+    tiles = ((T + bn - 1) / bn) * b.m_tiles;
     p->prof.begin(MOE_STAGE_SHARED_DOWN, s);
-    if (launch_gemm<KIND_BF16, EPI_F32>(p, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
+    if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
       return MOE_ERR_CUDA;
     p->prof.end(s);
   }
   // a9: weighted combine with the shared output
   p->prof.begin(MOE_STAGE_COMBINE, s);
-  combine_kernel<<<T, 128, k * 8, s>>>(O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
+  combine_kernel<<<dim3(T, (d + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
+      O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
   p->prof.end(s);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   p->last_T = T;
+  p->last_bn = bn;
   return MOE_OK;
 }
 
@@ -565,6 +588,20 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int option, int value) {
     case MOE_OPT_PREFETCH_B:
       p->pf_b = value != 0;
       return MOE_OK;
+    case MOE_OPT_TILE_N:
+      if (value != 0 && value != kBNSmall && value != kBN) return MOE_ERR_INVALID_ARG;
+      p->tile_n_opt = value;
+      return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t moe_plan_get_option(moe_plan_t p, int option, int* value) {
+  if (!p || !value) return MOE_ERR_INVALID_ARG;
+  switch (option) {
+    case MOE_OPT_PREFETCH_DIST: *value = p->pf_dist; return MOE_OK;
+    case MOE_OPT_PREFETCH_B: *value = p->pf_b; return MOE_OK;
+    case MOE_OPT_TILE_N: *value = p->last_bn; return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
 }
@@ -602,9 +639,9 @@ moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes
   size_t off, n;
   switch (which) {
     case 0: off = p->o_xq; n = A * p->d; break;
-    case 1: off = p->o_xs; n = (A / kBN + p->E + 1) * (p->d / 128) * SF_TILE_BYTES; break;
+    case 1: off = p->o_xs; n = (A / kBNMin + p->E + 1) * (p->d / 128) * SF_TILE_BYTES; break;
     case 2: off = p->o_hq; n = A * p->I; break;
-    case 3: off = p->o_hs; n = (A / kBN + p->E + 1) * (p->I / 128) * SF_TILE_BYTES; break;
+    case 3: off = p->o_hs; n = (A / kBNMin + p->E + 1) * (p->I / 128) * SF_TILE_BYTES; break;
     case 4: off = p->o_O; n = A * p->d * 2; break;
     case 5: off = p->o_ys; n = T * p->d * 4; break;
     case 6: off = p->o_logits; n = T * p->E * 4; break;

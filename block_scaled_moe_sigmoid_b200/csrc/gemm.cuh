@@ -24,8 +24,8 @@
 // Roles (384 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
 // scales), warp 10 loads the token rows (one TMA box, plus a bulk copy of their scales),
 // warp 11 copies each stage's scale factors into TMEM (KIND_MX), warp 1 owns TMEM and one
-// lane issues the MMAs, warps 2..9 run the epilogue (lane quarter = warp % 4).  The two
-// producers fill the same stage independently.
+// lane issues the MMAs, two K tiles per round, warps 2..9 run the epilogue (lane quarter =
+// warp % 4).  The producers and the scale warp complete the same stage independently.
 #pragma once
 #include "ptx.cuh"
 #include "tiling.cuh"
@@ -70,7 +70,7 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN_MAX * 128;
   static constexpr int SFA_BYTES = KIND == KIND_MX ? 1024 : 0;
   static constexpr int SFB_ATOMS = (BN_MAX + 127) / 128;
-  static constexpr int SFB_BYTES = KIND == KIND_MX ? SFB_ATOMS * 512 : 0;
+  static constexpr int SFB_BYTES = KIND == KIND_MX ? 1024 : 0;   // room for two 512 B atoms
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int A_TX = KIND == KIND_MX ? BM * BK / 2 : BM * BK * 2;  // global bytes
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
@@ -156,8 +156,7 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* ctrl = smem + STAGES * C::STAGE_BYTES;
   uint64_t* full_bar = (uint64_t*)ctrl;
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* sf_ready = empty_bar + STAGES;       // scale factors of the stage are in TMEM
-  uint64_t* sf_full = sf_ready + STAGES;         // scale blocks of the stage are in smem
+  uint64_t* sf_full = empty_bar + STAGES;        // scale blocks of the stage are in smem
   uint64_t* acc_full = sf_full + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain_bar = acc_empty + 1;
@@ -170,9 +169,10 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(full_bar + s), 2);  // one arrival per producer warp
+      // one arrival per producer warp, plus (KIND_MX) the scale warp's commit once the
+      // stage's scale factors are in TMEM: a full stage is ready for the MMAs as it stands
+      mbar_init(smem_u32(full_bar + s), KIND == KIND_MX ? 3 : 2);
       mbar_init(smem_u32(empty_bar + s), 1);
-      mbar_init(smem_u32(sf_ready + s), 1);
       mbar_init(smem_u32(sf_full + s), 2);   // weight-scale and token-scale copies
     }
     mbar_init(smem_u32(acc_full), 1);
@@ -297,8 +297,9 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------- scale factors -> TMEM
     // tcgen05.cp of each stage's scale atoms into that stage's TMEM buffer, off the MMA
     // thread's instruction stream, as soon as the small scale blocks land (their own
-    // barrier, ahead of the large tiles).  A buffer is rewritten only after the stage was
-    // released for refilling, i.e. after the MMAs that read it committed.
+    // barrier, ahead of the large tiles).  The copies' commit is the third arrival on the
+    // stage's full barrier.  A buffer is rewritten only after the stage was released for
+    // refilling, i.e. after the MMAs that read it committed.
     if (KIND == KIND_MX && lane == 0) {
       // no-swizzle descriptor of stage 0's A scale atoms (32 rows x 16 B, 128 B per 8 rows)
       const uint64_t sf_desc0 = smem_desc(smem_u32(smem) + C::A_BYTES + C::B_BYTES, 16, 128, 0);
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(384, 1)
           if (h1) tc_cp_32x128b_warpx4(tsf + 4, sfa_desc + (uint64_t)(512 >> 4));
           tc_cp_32x128b_warpx4(tsf + 8, sfb_desc);
           if (atoms > 1) tc_cp_32x128b_warpx4(tsf + 12, sfb_desc + (uint64_t)(512 >> 4));
-          tc_commit(smem_u32(sf_ready + stage));
+          tc_commit(smem_u32(full_bar + stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -351,15 +352,11 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
-          ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
-          if (ok && KIND == KIND_MX) ok = mbar_wait(smem_u32(sf_ready + stage), phase, args.status, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t a_desc = desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+        // the 8 MMAs (4 K-blocks x 2 halves) of the K tile held by smem stage st
+        auto issue_stage = [&](int st, uint32_t acc0) {
+          const uint64_t a_desc = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
           const uint64_t b_desc = a_desc + (uint64_t)(C::A_BYTES >> 4);
-          const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
-          const uint32_t acc0 = kt > 0 ? 1u : 0u;
+          const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * st;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
 #pragma unroll
@@ -375,8 +372,30 @@ __global__ void __launch_bounds__(384, 1)
                 mma_bf16(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], acc);
             }
           }
+        };
+        // Two K tiles per round: both stages' barriers are checked back to back and their 16
+        // MMAs issued in one run.  Each mbarrier wait costs the issuing thread about as much
+        // as one or two MMAs even when the stage has long landed, so pairing halves that
+        // overhead per MMA.  Each stage is still released as soon as its own MMAs commit.
+        for (int kt = 0; kt < args.k_tiles; kt += 2) {
+          const bool two = kt + 1 < args.k_tiles;
+          const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
+          const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
+          ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
+          if (ok && two) ok = mbar_wait(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_stage(stage, kt > 0 ? 1u : 0u);
           tc_commit(smem_u32(empty_bar + stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          if (two) {
+            issue_stage(stage2, 1u);
+            tc_commit(smem_u32(empty_bar + stage2));
+          }
+          stage = stage2;
+          phase = phase2;
+          if (two) {
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
         }
         if (!ok) break;
         tc_commit(smem_u32(acc_full));

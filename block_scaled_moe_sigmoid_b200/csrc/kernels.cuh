@@ -297,9 +297,14 @@ __global__ void topk_sigmoid_kernel(const float* __restrict__ z, int T, int E, i
 
 // ---------------------------------------------------------------- combine
 // y[t] = bf16( y_shared[t] + sum_j w[t][j] * O[inv[t][j]] ), fp32 sums in slot order.
-__global__ void combine_kernel(const __nv_bfloat16* __restrict__ O, const float* __restrict__ ys,
-                               const float* __restrict__ w, const int* __restrict__ inv, int T,
-                               int d, int k, __nv_bfloat16* __restrict__ y) {
+// Grid (T, ceil(d / 1024)): each thread owns 8 columns of one token; the k expert rows
+// are fetched four at a time so that several 16-byte loads are in flight per thread.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineCols = kCombineThreads * 8;
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_kernel(const __nv_bfloat16* __restrict__ O, const float* __restrict__ ys,
+                   const float* __restrict__ w, const int* __restrict__ inv, int T, int d, int k,
+                   __nv_bfloat16* __restrict__ y) {
   const int t = blockIdx.x;
   extern __shared__ int s_inv[];
   float* s_w = (float*)(s_inv + k);
@@ -308,37 +313,44 @@ __global__ void combine_kernel(const __nv_bfloat16* __restrict__ O, const float*
     s_w[j] = __ldg(w + (size_t)t * k + j);
   }
   __syncthreads();
-  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
-    float acc[8];
-    if (ys) {
-      const float4 a = __ldg((const float4*)(ys + (size_t)t * d + c));
-      const float4 b = __ldg((const float4*)(ys + (size_t)t * d + c + 4));
-      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
-    } else {
+  const int c = blockIdx.y * kCombineCols + threadIdx.x * 8;
+  if (c >= d) return;
+  float acc[8];
+  if (ys) {
+    const float4 a = __ldg((const float4*)(ys + (size_t)t * d + c));
+    const float4 b = __ldg((const float4*)(ys + (size_t)t * d + c + 4));
+    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+  } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  }
+  for (int j0 = 0; j0 < k; j0 += 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = j0 + q < k ? s_inv[j0 + q] : -1;
+      v[q] = p >= 0 ? __ldg((const uint4*)(O + (size_t)p * d + c)) : make_uint4(0, 0, 0, 0);
     }
-    for (int j = 0; j < k; ++j) {
-      const int p = s_inv[j];
-      if (p < 0) continue;
-      const uint4 v = __ldg((const uint4*)(O + (size_t)p * d + c));
-      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-      const float wj = s_w[j];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (j0 + q >= k || s_inv[j0 + q] < 0) continue;
+      const uint32_t wv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+      const float wj = s_w[j0 + q];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         acc[2 * i] = fmaf(wj, __uint_as_float(wv[i] << 16), acc[2 * i]);
         acc[2 * i + 1] = fmaf(wj, __uint_as_float(wv[i] & 0xFFFF0000u), acc[2 * i + 1]);
       }
     }
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-      o[i] = *(const uint32_t*)&p2;
-    }
-    *(uint4*)(y + (size_t)t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    o[i] = *(const uint32_t*)&p2;
+  }
+  *(uint4*)(y + (size_t)t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ---------------------------------------------------------------- weight packing (setup)

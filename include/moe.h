@@ -178,9 +178,18 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
 /* ---- tuning options ----------------------------------------------------------------
  * MOE_OPT_PREFETCH_DIST: the routed grouped GEMMs prefetch their weight tiles into L2
  *   this many K tiles ahead of the shared-memory loads (0..64, 0 = off).
- * MOE_OPT_PREFETCH_B: accepted and ignored (reserved). */
-enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1 };
+ * MOE_OPT_PREFETCH_B: accepted and ignored (reserved).
+ * MOE_OPT_TILE_N: token rows per grouped-GEMM tile.  0 (default) picks per call: 32 rows
+ *   (5-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure weight
+ *   stream, else 160 rows (4 stages).  32 or 160 forces one configuration; any other
+ *   value is MOE_ERR_INVALID_ARG.  Results do not depend on it beyond fp32 summation
+ *   order, which is the same (the K loop runs in the same order in both).
+ * moe_plan_get_option reads an option back (host int); for MOE_OPT_TILE_N it returns the
+ * tile rows that the last moe_forward on this plan used (0 before the first call), which
+ * fixes the tile-major layout of the token-side scale blocks (debug buffers 1 and 3). */
+enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1, MOE_OPT_TILE_N = 2 };
 moe_status_t moe_plan_set_option(moe_plan_t plan, int option, int value);
+moe_status_t moe_plan_get_option(moe_plan_t plan, int option, int* value);
 
 /* ---- per-stage timing ---------------------------------------------------------------
  * With profiling on, every stage of moe_route / moe_forward is bracketed by two CUDA

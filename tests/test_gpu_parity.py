@@ -150,9 +150,11 @@ def _stage_checks(case, idx, w):
     x = case.x_np()
     xq_ref, xs_ref = mx.quantize_mx(x, "e4m3")
     xq = case.plan.debug_tensor(0, torch.uint8, (A, wl.d)).cpu().numpy()
+    bn = api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_TILE_N)
+    assert bn in (32, 160)
     ptr, nbytes = api.moe_debug_buffer(case.plan.handle, 1)
     xs = decode_tile_major_scales(case.plan.debug_tensor(1, torch.uint8, (nbytes,)).cpu().numpy(),
-                                  counts, wl.d // 128)
+                                  counts, wl.d // 128, bn)
     assert np.array_equal(xq, xq_ref[perm_tok])
     assert np.array_equal(xs, xs_ref[perm_tok])
     # GLU output (MXFP8): decoded values agree up to one E4M3 step where fp32 and fp64
@@ -160,7 +162,7 @@ def _stage_checks(case, idx, w):
     hq = case.plan.debug_tensor(2, torch.uint8, (A, wl.I)).cpu().numpy()
     ptr, nbytes = api.moe_debug_buffer(case.plan.handle, 3)
     hs = decode_tile_major_scales(case.plan.debug_tensor(3, torch.uint8, (nbytes,)).cpu().numpy(),
-                                  counts, wl.I // 128)
+                                  counts, wl.I // 128, bn)
     H = mx.dequantize_mx(hq, hs, "e4m3")
     X = mx.dequantize_mx(xq_ref, xs_ref, "e4m3")
     worst, mism = 0.0, 0
@@ -209,6 +211,28 @@ def test_layer_hot_experts_span_several_tiles():
     bias[[3, 7, 11, 12]] = 40.0
     case = Case(wl, bias=bias)
     _check_layer(case, stage_checks=True)
+
+
+def test_layer_tile_configs_agree():
+    """Both grouped-GEMM tile configurations (32-row tiles with a 5-stage pipeline, 160-row
+    tiles with 4 stages) on one input whose hot experts span several tiles in each (400
+    rows: 13 tiles of <= 32 rows, 3 of <= 160): each matches the oracle, and the two give
+    the same bytes because the K loop runs in the same order."""
+    wl = synth.custom(seed=11, T=400, d=256, E=16, k=4, I=128, I_shared=128)
+    bias = torch.zeros(16)
+    bias[[1, 5, 6, 14]] = 40.0
+    case = Case(wl, bias=bias)
+    outs = []
+    for bn in (32, 160):
+        api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, bn)
+        _check_layer(case, stage_checks=True)
+        assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_TILE_N) == bn
+        idx, w = case.plan.route(case.x, case.W_r, case.bias)
+        outs.append(case.plan.forward(case.x, idx, w, case.experts, case.shared).cpu())
+    assert torch.equal(outs[0], outs[1])
+    api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 0)
+    with pytest.raises(api.MoeError):
+        api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 64)
 
 
 def test_layer_dense_mixture_k_equals_e():
