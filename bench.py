@@ -31,7 +31,7 @@ UNIT = "tokens/s"
 # workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` of this
 # kernel version (profiles/dram_gemm_k3_prefill_t8192.md).  None whenever the kernel
 # has changed since that capture.
-GATE_UP_TRAFFIC_BYTES = {8192: 24714007552 + 412475648}
+GATE_UP_TRAFFIC_BYTES = {8192: 24134107648 + 412293120}
 
 
 def parse():
@@ -233,6 +233,8 @@ def run_ours(args, rank, world, local_rank):
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} in the timed region")
     launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_ROUTER_SPLIT) > 1:
+        launches += stages["router_gemm"][1]   # the K-split partial sum
 
     # ---- end to end through the public API with host buffers
     e2e = None

@@ -44,7 +44,8 @@ SIGNATURES = {
 
 STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "gate_up_glu",
           "down", "shared_gate_up", "shared_down", "combine"]
-# kernel launches per recorded stage instance
+# kernel launches per recorded stage instance (router_gemm: +1 for the partial-sum kernel
+# when moe_plan_get_option(MOE_OPT_ROUTER_SPLIT) > 1)
 STAGE_KERNELS = {"permute": 3}
 
 
@@ -203,7 +204,7 @@ def moe_debug_buffer(plan, which):
     return p.value, n.value
 
 
-MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B, MOE_OPT_TILE_N = 0, 1, 2
+MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B, MOE_OPT_TILE_N, MOE_OPT_ROUTER_SPLIT = 0, 1, 2, 3
 
 
 def moe_plan_set_option(plan, option, value):

@@ -26,6 +26,7 @@ constexpr int kBNMin = kBNSmall;   // workspace sizing: the most tiles either co
 constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
 constexpr int kRouterStages = 3;
+constexpr int kRouterMaxCtas = 256;   // bound on split router tiles (sizes the partials)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -119,6 +120,7 @@ struct moe_plan_s {
   int pf_dist = 0, pf_b = 0;  // GEMM L2 prefetch (moe_plan_set_option)
   int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
   int last_bn = 0;            // token rows per tile in the last moe_forward
+  int last_ksplit = 0;        // router K splits in the last moe_route
   // token rows per GEMM tile for a call with T tokens
   int tile_rows(int T) const {
     if (tile_n_opt) return tile_n_opt;
@@ -127,7 +129,7 @@ struct moe_plan_s {
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
-  size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits,
+  size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
       o_planes, o_xq, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
   int tokens_per_chunk() const { return kPermThreads; }
   int nchunks(int T) const { return (T + kPermThreads - 1) / kPermThreads; }
@@ -147,6 +149,8 @@ static void carve(moe_plan_s* p) {
   p->o_perm = take(A * 4);
   p->o_inv = take(A * 4);
   p->o_logits = take((size_t)p->T_max * p->E * 4);
+  // K-split router partials: ksplit * ceil(T/128) * ceil(E/128) <= kRouterMaxCtas tiles
+  p->o_zpart = take((size_t)kRouterMaxCtas * kRouterBN * 128 * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
   p->o_xq = take(A * p->d);
   // token-side scale blocks, tile-major: at most A / bn + E group-tiles
@@ -354,15 +358,30 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   ra.m_tiles = (E + 127) / 128;
   ra.bias = bias;
   ra.z = z;
+  ra.zpart = p->at<float>(p->o_zpart);
   ra.status = p->at<unsigned int>(p->o_status);
   {
+    // Split K when the expert x token tiles would fill less than half the SMs, so that
+    // the plane reads (3 x E x d bf16) spread over the whole GPU.
+    const int chains = d / 64;
+    const int base_tiles = ((T + kRouterBN - 1) / kRouterBN) * ra.m_tiles;
+    const int cap = std::min(p->num_sms, kRouterMaxCtas);
+    int ksplit = 1;
+    if (2 * base_tiles <= cap) ksplit = std::min(chains, cap / base_tiles);
+    ra.chains_per = (chains + ksplit - 1) / ksplit;
+    ra.ksplit = (chains + ra.chains_per - 1) / ra.chains_per;
+    p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
     static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RC::SMEM_BYTES);
     if (attr != cudaSuccess) return MOE_ERR_CUDA;
-    const int tiles = ((T + kRouterBN - 1) / kRouterBN) * ra.m_tiles;
+    const int tiles = base_tiles * ra.ksplit;
     p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
     kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
+    if (ra.ksplit > 1) {
+      const long long n = (long long)T * E;
+      router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ra.zpart, ra.ksplit, bias, T, E, z);
+    }
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
@@ -602,6 +621,7 @@ moe_status_t moe_plan_get_option(moe_plan_t p, int option, int* value) {
     case MOE_OPT_PREFETCH_DIST: *value = p->pf_dist; return MOE_OK;
     case MOE_OPT_PREFETCH_B: *value = p->pf_b; return MOE_OK;
     case MOE_OPT_TILE_N: *value = p->last_bn; return MOE_OK;
+    case MOE_OPT_ROUTER_SPLIT: *value = p->last_ksplit; return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
 }

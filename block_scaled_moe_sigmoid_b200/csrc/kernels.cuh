@@ -257,6 +257,27 @@ __global__ void perm_place_kernel(const int* __restrict__ idx, int T, int k, int
 }
 
 // ---------------------------------------------------------------- top-k
+// K-split router logits: z[t][e] = (sum over s, in order, of zpart[s][t][e]) + bias[e].
+// One thread per logit; the partials are fetched eight at a time so that the loads
+// overlap, and added in split order.
+__global__ void router_reduce_kernel(const float* __restrict__ zpart, int nsplit,
+                                     const float* __restrict__ bias, int T, int E, float* __restrict__ z) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long n = (long long)T * E;
+  if (i >= n) return;
+  float v = 0.0f;
+  for (int s0 = 0; s0 < nsplit; s0 += 8) {
+    float p[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = s0 + q < nsplit ? __ldg(zpart + (size_t)(s0 + q) * n + i) : 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (s0 + q < nsplit) v = (s0 + q == 0) ? p[q] : v + p[q];
+  }
+  if (bias) v += __ldg(bias + (int)(i % E));
+  z[i] = v;
+}
+
 // One warp per token: k rounds of a warp arg-max over the logits (descending value,
 // lower index on ties), then sigmoid weights renormalised to sum 1.
 __global__ void topk_sigmoid_kernel(const float* __restrict__ z, int T, int E, int k,

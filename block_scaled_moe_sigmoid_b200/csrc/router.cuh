@@ -8,8 +8,12 @@
 // add each partial into fp32 registers (round-to-nearest).  Two partial buffers let the
 // tensor core run the next chain while the last one is drained.
 //
-// Tile: 128 experts (MMA M = lanes) x up to RBN tokens (MMA N = columns).  Roles as in
-// gemm.cuh: warp 0 loads (TMA), warp 1 issues MMAs, warps 2..9 drain and store.
+// Tile: 128 experts (MMA M = lanes) x up to RBN tokens (MMA N = columns) x a range of
+// 64-column chains.  With few tokens (decode) the expert x token tiles alone would occupy
+// a handful of SMs, so K is split: split s covers chains [s * chains_per, ...) and writes
+// its fp32 partial to zpart[s]; the top-k kernel adds the partials in split order and the
+// bias.  Roles as in gemm.cuh: warp 0 loads (TMA), warp 1 issues MMAs, warps 2..9 drain
+// and store.
 #pragma once
 #include "ptx.cuh"
 
@@ -17,11 +21,30 @@ namespace moe {
 
 struct RouterArgs {
   int T, d, E;
-  int m_tiles;  // ceil(E / 128)
+  int m_tiles;     // ceil(E / 128)
+  int ksplit;      // K splits (1: no split)
+  int chains_per;  // 64-column chains per split
   const float* bias;
-  float* z;     // [T][E]
+  float* z;        // [T][E] (ksplit == 1)
+  float* zpart;    // [ksplit][T][E] partials without bias (ksplit > 1)
   unsigned int* status;
 };
+
+struct RouterTile {
+  int mt, row0, split, c0, c1;
+};
+__device__ __forceinline__ RouterTile router_tile(const RouterArgs& a, int rbn, int t) {
+  const int n_tok_tiles = (a.T + rbn - 1) / rbn;
+  const int per_split = n_tok_tiles * a.m_tiles;
+  RouterTile r;
+  r.split = t / per_split;
+  const int rest = t - r.split * per_split;
+  r.mt = rest % a.m_tiles;
+  r.row0 = (rest / a.m_tiles) * rbn;
+  r.c0 = r.split * a.chains_per;
+  r.c1 = min(a.d / 64, r.c0 + a.chains_per);
+  return r;
+}
 
 template <int RBN, int STAGES>
 struct RouterCfg {
@@ -52,9 +75,8 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chains = args.d / 64;
   const int n_tok_tiles = (args.T + RBN - 1) / RBN;
-  const int num_tiles = n_tok_tiles * args.m_tiles;
+  const int num_tiles = n_tok_tiles * args.m_tiles * args.ksplit;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -87,10 +109,11 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const int mt = t % args.m_tiles, row0 = (t / args.m_tiles) * RBN;
+      const RouterTile rt = router_tile(args, RBN, t);
+      const int mt = rt.mt, row0 = rt.row0;
       const int n_mma = (min(RBN, args.T - row0) + 15) & ~15;
       const int nB = (n_mma + 31) >> 5;
-      for (int c = 0; c < chains; ++c) {
+      for (int c = rt.c0; c < rt.c1; ++c) {
         if (lane == 0) ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -117,10 +140,11 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       const uint64_t desc0 = smem_desc(smem_u32(smem), 16, 1024, 2);  // stage 0, plane 0
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int row0 = (t / args.m_tiles) * RBN;
+        const RouterTile rt = router_tile(args, RBN, t);
+        const int row0 = rt.row0;
         const int n_mma = (min(RBN, args.T - row0) + 15) & ~15;
         const uint32_t idesc = idesc_bf16(128, n_mma);
-        for (int c = 0; c < chains; ++c, ++g) {
+        for (int c = rt.c0; c < rt.c1; ++c, ++g) {
           const uint32_t b = g & 1, pph = (g >> 1) & 1;
           ok = mbar_wait(smem_u32(pempty + b), pph ^ 1, args.status, abort_flag);
           if (!ok) break;
@@ -152,7 +176,8 @@ __global__ void __launch_bounds__(320, 1)
     uint32_t g = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const int mt = t % args.m_tiles, row0 = (t / args.m_tiles) * RBN;
+      const RouterTile rt = router_tile(args, RBN, t);
+      const int mt = rt.mt, row0 = rt.row0;
       const int n_valid = min(RBN, args.T - row0);
       const int nchunks = ((n_valid + 15) & ~15) >> 4;
       constexpr int MYCH = RBN / 32;  // this warp's chunks of 16 columns: cs*MYCH .. cs*MYCH+MYCH-1
@@ -161,7 +186,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < MYCH; ++i)
 #pragma unroll
         for (int j = 0; j < 16; ++j) accv[i][j] = 0.0f;
-      for (int c = 0; c < chains; ++c, ++g) {
+      for (int c = rt.c0; c < rt.c1; ++c, ++g) {
         const uint32_t b = g & 1, pph = (g >> 1) & 1;
         if (lane == 0) ok = mbar_wait(smem_u32(pfull + b), pph, args.status, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -185,13 +210,15 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) break;
       const int e = mt * 128 + q * 32 + lane;
       if (e < args.E) {
-        const float bias = args.bias ? __ldg(args.bias + e) : 0.0f;
+        const bool split = args.ksplit > 1;
+        const float bias = (!split && args.bias) ? __ldg(args.bias + e) : 0.0f;
+        float* out = split ? args.zpart + (size_t)rt.split * args.T * args.E : args.z;
 #pragma unroll
         for (int i = 0; i < MYCH; ++i)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = (cs * MYCH + i) * 16 + j;
-            if (n < n_valid) args.z[(size_t)(row0 + n) * args.E + e] = accv[i][j] + bias;
+            if (n < n_valid) out[(size_t)(row0 + n) * args.E + e] = split ? accv[i][j] : accv[i][j] + bias;
           }
       }
     }

@@ -184,10 +184,14 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  *   stream, else 160 rows (4 stages).  32 or 160 forces one configuration; any other
  *   value is MOE_ERR_INVALID_ARG.  Results do not depend on it beyond fp32 summation
  *   order, which is the same (the K loop runs in the same order in both).
+ * MOE_OPT_ROUTER_SPLIT (read only): the number of K splits the last moe_route used for
+ *   the router GEMM (1 = none).  With few tokens the router splits d over up to one
+ *   CTA per SM and adds the fp32 partials in split order (plus the bias) in one more
+ *   kernel, so that call launches 4 kernels instead of 3.
  * moe_plan_get_option reads an option back (host int); for MOE_OPT_TILE_N it returns the
  * tile rows that the last moe_forward on this plan used (0 before the first call), which
  * fixes the tile-major layout of the token-side scale blocks (debug buffers 1 and 3). */
-enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1, MOE_OPT_TILE_N = 2 };
+enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1, MOE_OPT_TILE_N = 2, MOE_OPT_ROUTER_SPLIT = 3 };
 moe_status_t moe_plan_set_option(moe_plan_t plan, int option, int value);
 moe_status_t moe_plan_get_option(moe_plan_t plan, int option, int* value);
 
