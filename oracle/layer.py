@@ -30,6 +30,12 @@ Readings (the pages leave these open):
       rounded to bf16 (the precision of the operand of the second product).
   R16 Output: y = y_shared + sum_j w_j * o_j accumulated in fp64, then rounded
       once to bf16 (ties to even).
+  R17 Second GLU (an option, not the Kimi default): the clamped SwiGLU that
+      "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, routed-experts
+      row, describes for gpt-oss.  The gate is clamped from above at 7.0, the
+      linear branch to [-7, 7], and a = (u_c + 1) * g_c * sigmoid(1.702 g_c).
+      Reading: "gate" is the first projection g and "linear branch" the second u.
+      The plan's activation applies to every GLU of the layer, routed and shared.
 """
 import numpy as np
 
@@ -41,7 +47,20 @@ def silu(g):
     return g / (1.0 + np.exp(-g))
 
 
-ACTIVATIONS = {"silu": silu}
+def glu_silu(g, u):
+    """SiLU-GLU (R11): silu(g) * u."""
+    return silu(g) * np.asarray(u, dtype=np.float64)
+
+
+def glu_clamped_swiglu(g, u, limit=7.0, alpha=1.702):
+    """Clamped SwiGLU (R17): (clip(u, -7, 7) + 1) * g_c * sigmoid(1.702 g_c), g_c = min(g, 7)."""
+    gc = np.minimum(np.asarray(g, dtype=np.float64), limit)
+    uc = np.clip(np.asarray(u, dtype=np.float64), -limit, limit)
+    return (uc + 1.0) * gc / (1.0 + np.exp(-alpha * gc))
+
+
+# GLU activations by name: a = glu(g, u)
+ACTIVATIONS = {"silu": glu_silu, "clamped_swiglu": glu_clamped_swiglu}
 
 
 def quantize_expert(W_gate, W_up, W_down):
@@ -64,10 +83,10 @@ def decode_expert(q):
 
 
 def expert_hidden(X, Wg, Wu, act="silu"):
-    """a = act(X Wg^T) * (X Wu^T) in fp64 (R11, R13).  X: [M, d] exact values."""
+    """a = glu(X Wg^T, X Wu^T) in fp64 (R11, R13, R17).  X: [M, d] exact values."""
     g = X @ Wg.T
     u = X @ Wu.T
-    return ACTIVATIONS[act](g) * u
+    return ACTIVATIONS[act](g, u)
 
 
 def expert_forward(X, Wg, Wu, Wd, act="silu"):

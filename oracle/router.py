@@ -20,6 +20,13 @@ Readings (the pages leave these open):
      The output order is the selection order.
   R9 The "16th/17th gap" of a token is sigmoid(z_(k)) - sigmoid(z_(k+1)) in fp64
      (z_(i) is the i-th largest logit); it is +inf when k == E.
+  R10 Select-only bias (second mode).  The same rows call b a per-expert
+     *selection* bias, and the raw config of "Kimi K3" (llm-atlas) has
+     topk_method noaux_tc.  The plainest reading of both: experts are chosen
+     by z + b, while the weights come from the unbiased s = sigmoid(z).  Ties
+     and the gap (R7, R9) then apply to the key z + b.  The key is formed in
+     the precision of the z passed in, so that a caller holding fp32 logits
+     takes the same integer decision as an fp32 kernel.
 """
 import numpy as np
 
@@ -59,19 +66,27 @@ def topk_select(z, k):
     return idx
 
 
-def route(z, k):
+def route(z, k, select_bias=None):
     """Selection, renormalised weights and the k/k+1 score gap (R7, R8, R9).
 
+    select_bias: None (any bias is already inside z, R6) or the [E] bias of the
+    select-only mode (R10): selection by z + b, weights from sigmoid(z).
     Returns (idx int32 [T,k], w fp64 [T,k], gap fp64 [T]).
     """
-    z = np.asarray(z, dtype=np.float64)
+    z_in = np.asarray(z)
+    if select_bias is None:
+        key = z_in
+    else:
+        key = z_in + np.asarray(select_bias, dtype=z_in.dtype)[None, :]
+    key = np.asarray(key, dtype=np.float64)
+    z = np.asarray(z_in, dtype=np.float64)
     T, E = z.shape
-    idx = topk_select(z, k)
+    idx = topk_select(key, k)
     s_sel = sigmoid(np.take_along_axis(z, idx.astype(np.int64), axis=1))
     w = s_sel / np.sum(s_sel, axis=1, keepdims=True)
     if k < E:
-        zs = -np.sort(-z, axis=1)
-        gap = sigmoid(zs[:, k - 1]) - sigmoid(zs[:, k])
+        ks = -np.sort(-key, axis=1)
+        gap = sigmoid(ks[:, k - 1]) - sigmoid(ks[:, k])
     else:
         gap = np.full(T, np.inf)
     return idx, w, gap

@@ -175,3 +175,49 @@ def test_relative_error_definition():
     assert abs(r[0, 0] - 0.01 / max(1.0, rms)) < 1e-15
     assert abs(r[0, 2] - 0.001 / rms) < 1e-15
     assert abs(nw[0] - math.sqrt(0.01 ** 2 + 0.001 ** 2) / math.sqrt(5.25)) < 1e-15
+
+
+# ------------------------------------------------------------------ clamped SwiGLU (R17)
+def test_clamped_swiglu_inside_the_clamps_is_scaled_torch_silu():
+    """Inside the clamps, (u + 1) * g * sigmoid(1.702 g) equals (u + 1) * silu(1.702 g) / 1.702.
+    torch's silu (a library routine) pins the sigmoid factor and which operand is the gate."""
+    rng = np.random.default_rng(11)
+    g = rng.uniform(-12.0, 7.0, 4096)
+    u = rng.uniform(-7.0, 7.0, 4096)
+    a = layer.ACTIVATIONS["clamped_swiglu"](g, u)
+    ref = (torch.from_numpy(u) + 1.0) * F.silu(1.702 * torch.from_numpy(g)) / 1.702
+    assert np.allclose(a, ref.numpy(), rtol=1e-14, atol=1e-300)
+    # a gate/linear swap fails the pin (the two operands play different roles)
+    assert not np.allclose(layer.ACTIVATIONS["clamped_swiglu"](u, g), ref.numpy(), rtol=1e-6)
+
+
+def test_clamped_swiglu_clamps_and_zeros():
+    f = layer.ACTIVATIONS["clamped_swiglu"]
+    g = np.array([7.0, 7.5, 100.0, 1e30])
+    u = np.array([0.3, 0.3, 0.3, 0.3])
+    assert np.all(f(g, u) == f(np.full(4, 7.0), u))          # gate clamped from above at 7
+    assert f(-50.0, 1.0) != f(-7.0, 1.0)                      # ... but not from below
+    assert f(2.0, 9.0) == f(2.0, 7.0) and f(2.0, -9.0) == f(2.0, -7.0)   # linear branch to [-7, 7]
+    assert f(3.0, -1.0) == 0.0 and f(0.0, 5.0) == 0.0        # (u + 1) and g factors
+    assert f(2.0, -7.0) == -6.0 * f(2.0, 0.0)                 # (u + 1) is linear in u
+
+
+def test_single_expert_clamped_swiglu_torch():
+    """E = k = 1 with the clamped SwiGLU reduces to one dense MLP (torch float64 GEMMs)."""
+    rng = np.random.default_rng(12)
+    x = _bf16(rng.standard_normal((16, 128)) * 3.0)
+    Ws = _experts(rng, 1, 128, 64)
+    Ws = [tuple(W * 40.0 for W in Ws[0])]       # large pre-activations reach both clamps
+    idx = np.zeros((16, 1), np.int32)
+    w = np.ones((16, 1))
+    y = layer.moe_layer(x, idx, w, lambda e: Ws[0], act="clamped_swiglu")
+    xq, xs = mx.quantize_mx(x, "e4m3")
+    X = torch.from_numpy(mx.dequantize_mx(xq, xs, "e4m3"))
+    Wg, Wu, Wd = (torch.from_numpy(a) for a in Ws[0])
+    g, u = F.linear(X, Wg), F.linear(X, Wu)
+    assert (g > 7).any() and (u.abs() > 7).any()
+    gc, uc = g.clamp(max=7.0), u.clamp(-7.0, 7.0)
+    a = (uc + 1.0) * F.silu(1.702 * gc) / 1.702
+    hq, hs = mx.quantize_mx(a.numpy(), "e4m3")
+    o = F.linear(torch.from_numpy(mx.dequantize_mx(hq, hs, "e4m3")), Wd).numpy()
+    assert np.allclose(y, mx.bf16_round(o), rtol=2 ** -7, atol=0)

@@ -1,6 +1,7 @@
 """Pins for the oracle's router (oracle/router.py) and permutation (oracle/permute.py):
 brute force on tiny inputs, the tie rule, and the routing invariants."""
 import itertools
+import math
 
 import numpy as np
 
@@ -111,3 +112,53 @@ def test_config_closed_forms():
     assert abs(routed / 1e12 - float(cfg["total_params_trillion"])) < 0.1
     assert abs(100.0 * k / E - float(cfg["active_share_percent"])) < 0.05
     assert int(cfg["hidden_size"]) == 2 * dl
+
+
+# ------------------------------------------------------------------ select-only bias (R10)
+def test_select_only_bias_brute_force():
+    """Selection by z + b (full sort, lower index on ties), weights from sigmoid(z)."""
+    rng = np.random.default_rng(21)
+    T, E, k = 7, 12, 4
+    z = rng.standard_normal((T, E))
+    b = rng.standard_normal(E)
+    b[3] = b[5] = 0.25
+    z[:, 3] = z[:, 5] = 0.1          # an exact tie on the key, broken by the index
+    idx, w, gap = router.route(z, k, select_bias=b)
+    for t in range(T):
+        key = [(-(z[t, e] + b[e]), e) for e in range(E)]
+        sel = [e for _, e in sorted(key)[:k]]
+        assert list(idx[t]) == sel
+        s = [1.0 / (1.0 + math.exp(-z[t, e])) for e in sel]
+        assert np.allclose(w[t], [v / sum(s) for v in s], rtol=1e-15, atol=0)
+        keys = sorted((z[t, e] + b[e] for e in range(E)), reverse=True)
+        g = 1.0 / (1.0 + math.exp(-keys[k - 1])) - 1.0 / (1.0 + math.exp(-keys[k]))
+        assert abs(gap[t] - g) <= 1e-15
+
+
+def test_select_only_agrees_with_logit_bias_on_selection():
+    rng = np.random.default_rng(22)
+    z = rng.standard_normal((50, 64))
+    b = rng.standard_normal(64)
+    i1, w1, _ = router.route(z, 8, select_bias=b)
+    i2, w2, _ = router.route(z + b[None, :], 8)
+    assert np.array_equal(i1, i2)                 # same key, same experts
+    assert not np.allclose(w1, w2)                # weights differ: sigmoid(z) vs sigmoid(z + b)
+    i0, w0, g0 = router.route(z, 8, select_bias=np.zeros(64))
+    i3, w3, g3 = router.route(z, 8)
+    assert np.array_equal(i0, i3) and np.array_equal(w0, w3) and np.array_equal(g0, g3)
+
+
+def test_select_only_key_in_fp32_when_given_fp32():
+    """The key is formed in the logits' own precision, so fp32 logits give fp32 decisions."""
+    z = np.array([[1.0, 1.0 + 2.0 ** -23]], dtype=np.float32)
+    b = np.array([2.0 ** -24, 0.0], dtype=np.float32)
+    # in fp32, 1 + 2^-24 rounds to 1 (ties to even): the keys are (1, 1 + 2^-23), expert 1 wins;
+    # in fp64 the keys would be (1 + 2^-24, 1 + 2^-23): expert 1 wins as well, so use a tie
+    z2 = np.array([[1.0 + 2.0 ** -23, 1.0]], dtype=np.float32)
+    b2 = np.array([0.0, 2.0 ** -23 + 2.0 ** -25], dtype=np.float32)
+    idx, _, _ = router.route(z2, 1, select_bias=b2)
+    # fp32: 1 + (2^-23 + 2^-25) rounds to 1 + 2^-23, a tie with expert 0, which wins (lower index)
+    assert idx[0, 0] == 0
+    idx64, _, _ = router.route(z2.astype(np.float64), 1, select_bias=b2.astype(np.float64))
+    assert idx64[0, 0] == 1                       # in fp64 the key of expert 1 is larger
+    assert router.route(z, 1, select_bias=b)[0][0, 0] == 1
