@@ -118,9 +118,12 @@ struct moe_plan_s {
   int num_sms = 148;
   int last_T = 0;
   int pf_dist = 0, pf_b = 0;  // GEMM L2 prefetch (moe_plan_set_option)
+  int act = MOE_ACT_SILU_GLU;
+  int bias_mode = MOE_BIAS_LOGIT;
   int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
   int last_bn = 0;            // token rows per tile in the last moe_forward
   int last_ksplit = 0;        // router K splits in the last moe_route
+  size_t zpart_floats = 0;    // capacity of the router partials
   // token rows per GEMM tile for a call with T tokens
   int tile_rows(int T) const {
     if (tile_n_opt) return tile_n_opt;
@@ -149,8 +152,10 @@ static void carve(moe_plan_s* p) {
   p->o_perm = take(A * 4);
   p->o_inv = take(A * 4);
   p->o_logits = take((size_t)p->T_max * p->E * 4);
-  // K-split router partials: ksplit * ceil(T/128) * ceil(E/128) <= kRouterMaxCtas tiles
-  p->o_zpart = take((size_t)kRouterMaxCtas * kRouterBN * 128 * 4);
+  // K-split router partials [ksplit][T][E]: few tokens split up to kRouterMaxCtas tiles
+  // (ksplit * T * E <= kRouterMaxCtas * 128 * 128), many tokens split at most 3 ways
+  p->zpart_floats = std::max((size_t)kRouterMaxCtas * kRouterBN * 128, (size_t)3 * p->T_max * p->E);
+  p->o_zpart = take(p->zpart_floats * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
   p->o_xq = take(A * p->d);
   // token-side scale blocks, tile-major: at most A / bn + E group-tiles
@@ -194,6 +199,7 @@ static GemmArgs base_args(const moe_plan_s* p) {
   a.dense_rows = -1;
   a.pf_dist = p->pf_dist;
   a.pf_b = p->pf_b;
+  a.act = p->act;
   return a;
 }
 
@@ -241,13 +247,17 @@ moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared
                              moe_bias_mode_t bias_mode, int flags, moe_plan_t* out) {
   if (!out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
-  if (act != MOE_ACT_SILU_GLU || bias_mode != MOE_BIAS_LOGIT || flags != 0) return MOE_ERR_INVALID_ARG;
+  if ((act != MOE_ACT_SILU_GLU && act != MOE_ACT_CLAMPED_SWIGLU) ||
+      (bias_mode != MOE_BIAS_LOGIT && bias_mode != MOE_BIAS_SELECT_ONLY) || flags != 0)
+    return MOE_ERR_INVALID_ARG;
   if (T_max < 0 || d <= 0 || E <= 0 || k <= 0 || I <= 0 || I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (d % 128 || I % 128 || I_shared % 128 || k > E || k > 32 || E > 4096)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((long long)T_max * k > (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_plan_s* p = new moe_plan_s();
   p->T_max = T_max; p->d = d; p->E = E; p->k = k; p->I = I; p->Is = I_shared;
+  p->act = act;
+  p->bias_mode = bias_mode;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) {
     int sms = 0;
@@ -356,20 +366,37 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   ra.d = d;
   ra.E = E;
   ra.m_tiles = (E + 127) / 128;
-  ra.bias = bias;
+  // MOE_BIAS_SELECT_ONLY: z stays unbiased; the bias only enters the top-k key
+  const bool select_only = p->bias_mode == MOE_BIAS_SELECT_ONLY;
+  ra.bias = select_only ? nullptr : bias;
   ra.z = z;
   ra.zpart = p->at<float>(p->o_zpart);
   ra.status = p->at<unsigned int>(p->o_status);
   {
-    // Split K when the expert x token tiles would fill less than half the SMs, so that
-    // the plane reads (3 x E x d bf16) spread over the whole GPU.
+    // Split K (i) when the expert x token tiles would fill less than half the SMs, so that
+    // the plane reads (3 x E x d bf16) spread over the whole GPU, and (ii) otherwise by up
+    // to 3 when that evens out the last wave of the persistent grid (T=8192: 448 tiles on
+    // 148 SMs run 4 waves for 3.03 waves of work; split 3 runs 10 for 9.08).
     const int chains = d / 64;
     const int base_tiles = ((T + kRouterBN - 1) / kRouterBN) * ra.m_tiles;
     const int cap = std::min(p->num_sms, kRouterMaxCtas);
     int ksplit = 1;
-    if (2 * base_tiles <= cap) ksplit = std::min(chains, cap / base_tiles);
+    if (2 * base_tiles <= cap) {
+      ksplit = std::min(chains, cap / base_tiles);
+    } else {
+      double best = 0.0;
+      for (int sp = 1; sp <= 3 && chains / sp >= 16; ++sp) {
+        const long long units = (long long)base_tiles * sp;
+        const double eff = (double)units / (double)(((units + p->num_sms - 1) / p->num_sms) * p->num_sms);
+        if (eff > best + 0.03) { best = eff; ksplit = sp; }
+      }
+    }
     ra.chains_per = (chains + ksplit - 1) / ksplit;
     ra.ksplit = (chains + ra.chains_per - 1) / ra.chains_per;
+    if ((size_t)ra.ksplit * T * E > p->zpart_floats) {   // cannot happen with the sizing above
+      ra.ksplit = 1;
+      ra.chains_per = chains;
+    }
     p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
@@ -380,7 +407,7 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
     if (ra.ksplit > 1) {
       const long long n = (long long)T * E;
-      router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ra.zpart, ra.ksplit, bias, T, E, z);
+      router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ra.zpart, ra.ksplit, ra.bias, T, E, z);
     }
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
@@ -388,7 +415,8 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   if (set_smem_attrs() != cudaSuccess) return MOE_ERR_CUDA;
   const int wpb = 8;
   p->prof.begin(MOE_STAGE_TOPK, s);
-  topk_sigmoid_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * E * 4, s>>>(z, T, E, p->k, idx, w);
+  topk_sigmoid_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * E * 4, s>>>(
+      z, select_only ? bias : nullptr, T, E, p->k, idx, w);
   p->prof.end(s);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   p->last_T = T;

@@ -34,8 +34,8 @@ namespace moe {
 
 enum { KIND_MX = 0, KIND_BF16 = 1 };
 enum {
-  EPI_GLU_MX8 = 0,   // a = silu(gate) * up, requantised to MXFP8 along the channels
-  EPI_GLU_BF16 = 1,  // a = silu(gate) * up, stored as bf16
+  EPI_GLU_MX8 = 0,   // a = glu(gate, up), requantised to MXFP8 along the channels
+  EPI_GLU_BF16 = 1,  // a = glu(gate, up), stored as bf16
   EPI_BF16 = 2,      // D stored as bf16
   EPI_F32 = 3        // D stored as fp32
 };
@@ -60,6 +60,7 @@ struct GemmArgs {
   int pf_dist;          // L2 prefetch distance in k-tiles (0 = off), KIND_MX weights
   int pf_b;             // reserved
   const uint8_t* a_ptr; // KIND_MX: packed weights (base of the tile-major code array)
+  int act;              // GLU epilogues: MOE_ACT_SILU_GLU (0) or MOE_ACT_CLAMPED_SWIGLU (1)
 };
 
 template <int KIND, int BN_MAX, int STAGES>
@@ -127,6 +128,14 @@ __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, 
 }
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+// a = glu(g, u): act 0 SiLU-GLU; act 1 clamped SwiGLU, (clamp(u, -7, 7) + 1) * g_c *
+// sigmoid(1.702 g_c) with g_c = min(g, 7)
+__device__ __forceinline__ float glu_f(int act, float g, float u) {
+  if (act == 0) return silu_f(g) * u;
+  const float gc = fminf(g, 7.0f);
+  const float uc = fminf(fmaxf(u, -7.0f), 7.0f);
+  return (uc + 1.0f) * __fdividef(gc, 1.0f + __expf(-1.702f * gc));
+}
 
 // MXFP8 (E4M3) encoding of v with block scale exponent from the block's amax bits.
 __device__ __forceinline__ int mx_exp_e4m3(uint32_t amax_bits) {
@@ -428,7 +437,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(smem_u32(acc_empty));
       };
       if constexpr (EPI == EPI_GLU_MX8 || EPI == EPI_GLU_BF16) {
-        // a = silu(g) * u for this warp's chunks (c = sub + 2 i) straight out of TMEM;
+        // a = glu(g, u) for this warp's chunks (c = sub + 2 i) straight out of TMEM;
         // TMEM goes back to the MMA warp before the quantisation and stores.
         float a[CH / 2][16];
 #pragma unroll
@@ -440,7 +449,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld16(lane_base + BN_MAX + c * 16, u);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a[i][j] = silu_f(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+            for (int j = 0; j < 16; ++j) a[i][j] = glu_f(args.act, __uint_as_float(g[j]), __uint_as_float(u[j]));
           }
         }
         release_tmem();

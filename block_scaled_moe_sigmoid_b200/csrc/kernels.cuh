@@ -109,16 +109,34 @@ __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int 
   const uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
   const uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
   const int k_tiles = cols >> 7;
-  for (int j = 0; j < k; ++j) {
-    const int p = __ldg(inv + t * k + j);
-    if (p < 0 || p >= A_rows) continue;
-    uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
-    dst[0] = o0;
-    dst[1] = o1;
-    if ((l & 3) == 0) {
-      int gt, n;
-      row_tile(counts, offsets, tile_prefix, __ldg(idx + t * k + j), p, gt, n);
-      *(uint32_t*)(xs + ((size_t)gt * k_tiles + (b >> 2)) * SF_TILE_BYTES + sf_atom_offset(n)) = word;
+  const bool sc_lane = (l & 3) == 0;   // this lane writes the 4-block scale word
+  // four destinations at a time, so that their index loads and tile lookups overlap
+  for (int j0 = 0; j0 < k; j0 += 4) {
+    int pj[4], ej[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q;
+      pj[q] = j < k ? __ldg(inv + t * k + j) : -1;
+      ej[q] = (j < k && sc_lane) ? __ldg(idx + t * k + j) : 0;
+    }
+    size_t soff[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      soff[q] = 0;
+      if (sc_lane && pj[q] >= 0 && pj[q] < A_rows) {
+        int gt, n;
+        row_tile(counts, offsets, tile_prefix, ej[q], pj[q], gt, n);
+        soff[q] = ((size_t)gt * k_tiles + (b >> 2)) * SF_TILE_BYTES + sf_atom_offset(n);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = pj[q];
+      if (p < 0 || p >= A_rows) continue;
+      uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
+      dst[0] = o0;
+      dst[1] = o1;
+      if (sc_lane) *(uint32_t*)(xs + soff[q]) = word;
     }
   }
 }
@@ -280,14 +298,19 @@ __global__ void router_reduce_kernel(const float* __restrict__ zpart, int nsplit
 
 // One warp per token: k rounds of a warp arg-max over the logits (descending value,
 // lower index on ties), then sigmoid weights renormalised to sum 1.
-__global__ void topk_sigmoid_kernel(const float* __restrict__ z, int T, int E, int k,
-                                    int* __restrict__ idx_out, float* __restrict__ w_out) {
+// select_bias != NULL (select-only bias): the arg-max runs on the key z + b (fp32), the
+// weights still come from sigmoid(z).
+__global__ void topk_sigmoid_kernel(const float* __restrict__ z, const float* __restrict__ select_bias,
+                                    int T, int E, int k, int* __restrict__ idx_out,
+                                    float* __restrict__ w_out) {
   extern __shared__ float zs[];  // [warps][E]
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + w;
   if (t >= T) return;
   float* row = zs + (size_t)w * E;
-  for (int e = lane; e < E; e += 32) row[e] = __ldg(z + (size_t)t * E + e);
+  // row holds the selection key (z, or z + b in select-only mode)
+  for (int e = lane; e < E; e += 32)
+    row[e] = select_bias ? __ldg(z + (size_t)t * E + e) + __ldg(select_bias + e) : __ldg(z + (size_t)t * E + e);
   __syncwarp();
   float ssum = 0.0f, my_s = 0.0f;
   int my_i = -1;
@@ -304,7 +327,8 @@ __global__ void topk_sigmoid_kernel(const float* __restrict__ z, int T, int E, i
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    const float s = 1.0f / (1.0f + expf(-bv));
+    const float zsel = select_bias ? __ldg(z + (size_t)t * E + bi) : bv;
+    const float s = 1.0f / (1.0f + expf(-zsel));
     ssum += s;
     if (lane == r) { my_s = s; my_i = bi; }
     if (lane == 0) row[bi] = -INFINITY;

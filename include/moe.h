@@ -52,8 +52,21 @@ typedef enum {
   MOE_ERR_DEVICE_FAULT = 7       /* a kernel flagged bad input (e.g. expert id >= E) */
 } moe_status_t;
 
-typedef enum { MOE_ACT_SILU_GLU = 0 } moe_act_t;
-typedef enum { MOE_BIAS_LOGIT = 0 } moe_bias_mode_t;
+/* GLU activation of every expert of the layer, routed and shared: a = glu(g, u) with
+ * g = x Wg^T, u = x Wu^T.
+ *   MOE_ACT_SILU_GLU (default; the pages name SiTU-GLU but publish no formula):
+ *     a = g / (1 + exp(-g)) * u.
+ *   MOE_ACT_CLAMPED_SWIGLU: the gpt-oss expert of "Kimi K3.1 Pro vs gpt-oss-120b"
+ *     (archdiff), component table, routed-experts row.  g_c = min(g, 7),
+ *     u_c = clamp(u, -7, 7), a = (u_c + 1) * g_c / (1 + exp(-1.702 g_c)). */
+typedef enum { MOE_ACT_SILU_GLU = 0, MOE_ACT_CLAMPED_SWIGLU = 1 } moe_act_t;
+/* Router bias.
+ *   MOE_BIAS_LOGIT (default): z = x.W_r + b; selection and weights both come from z.
+ *   MOE_BIAS_SELECT_ONLY: the per-expert "selection bias" of the router row in the same
+ *     table, with topk_method noaux_tc from the raw config of "Kimi K3" (llm-atlas).
+ *     Experts are chosen by z + b, computed in fp32, with the same tie rule.  The weights
+ *     come from the unbiased s = sigmoid(z), and logits_opt receives z without b. */
+typedef enum { MOE_BIAS_LOGIT = 0, MOE_BIAS_SELECT_ONLY = 1 } moe_bias_mode_t;
 
 /* Packed MXFP4 expert weights (device pointers, all 256-byte aligned).
  *   Rows of gate and up are channel blocks of 128 interleaved as gate[0:128], up[0:128],
@@ -112,7 +125,8 @@ moe_status_t moe_quant_mxfp8(const void* x_bf16, int rows, int cols, uint8_t* q_
 /* ---- a2/a3: router --------------------------------------------------------------------
  * z = x . W_r + bias (fp32-accurate: W_r is split into three bf16 terms on the tensor
  * cores), s = sigmoid(z); per token the k largest z in descending order (lower expert
- * index on ties) and w_j = s_j / sum of the selected s.
+ * index on ties) and w_j = s_j / sum of the selected s.  With MOE_BIAS_SELECT_ONLY the
+ * bias enters only the selection key z + b (see moe_bias_mode_t).
  * x_bf16: device [T][d]; W_r: device fp32 [d][E]; bias: device fp32 [E] or NULL;
  * idx: device int32 [T][k]; w: device fp32 [T][k]; logits_opt: device fp32 [T][E] or
  * NULL (receives z).  Uses the plan workspace. */
@@ -151,8 +165,9 @@ moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int32_
 
 /* ---- a4..a9: the layer ----------------------------------------------------------------
  * y = bf16( shared(x) + sum_j w[t][j] * expert_{idx[t][j]}(x) ), where an expert is
- * down(silu(x Wg^T) * (x Wu^T)) on MXFP8 x and MXFP4 weights, its GLU output requantised
- * to MXFP8, and shared(x) = bf16(silu(x Wsg^T) * (x Wsu^T)) Wsd^T in bf16/fp32.
+ * down(glu(x Wg^T, x Wu^T)) on MXFP8 x and MXFP4 weights, its GLU output requantised
+ * to MXFP8, and shared(x) = bf16(glu(x Wsg^T, x Wsu^T)) Wsd^T in bf16/fp32 (glu: the
+ * plan's moe_act_t).
  * x_bf16: device [T][d]; idx/w: device [T][k] (e.g. from moe_route); experts: packed
  * weights; shared: NULL when the plan has I_shared = 0; y_bf16: device [T][d].
  * T = 0 is a no-op.  Uses the plan workspace (one call at a time per plan). */

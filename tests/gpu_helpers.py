@@ -73,18 +73,23 @@ class Case:
     """A workload: generator draws on `gen_device`, copied to the GPU for the kernels and
     to the CPU for the oracle."""
 
-    def __init__(self, wl, T=None, gen_device=None, bias=None):
+    def __init__(self, wl, T=None, gen_device=None, bias=None, act="silu", select_only=False,
+                 x_scale=1.0):
         self.wl = wl
+        self.act = act
+        self.select_only = select_only
         self.T = wl.T if T is None else T
         gd = wl.device if gen_device is None else gen_device
         self.gen_device = gd
         dev = "cuda"
-        self.x = synth.draw_x(wl, self.T, device=gd).to(dev)
+        self.x = (synth.draw_x(wl, self.T, device=gd) * x_scale).to(dev)   # x_scale: power of two
         W_r, b = synth.draw_router(wl, device=gd)
         if bias is not None:
             b = bias.to(torch.float32)
         self.W_r, self.bias = W_r.to(dev).contiguous(), b.to(dev).contiguous()
-        self.plan = api.Plan(max(self.T, 1), wl.d, wl.E, wl.k, wl.I, wl.I_shared)
+        self.plan = api.Plan(max(self.T, 1), wl.d, wl.E, wl.k, wl.I, wl.I_shared,
+                             act={"silu": api.MOE_ACT_SILU_GLU, "clamped_swiglu": api.MOE_ACT_CLAMPED_SWIGLU}[act],
+                             bias_mode=api.MOE_BIAS_SELECT_ONLY if select_only else api.MOE_BIAS_LOGIT)
         self.experts = api.Experts(wl.d, wl.I, wl.E)
         for e in range(wl.E):
             g, u, dn = (t.to(dev) for t in synth.draw_expert(wl, e, device=gd))
@@ -117,7 +122,11 @@ class Case:
         return tuple(t.float().cpu().numpy().astype(np.float64) for t in self.shared_w)
 
     def oracle_route(self):
-        z = router.router_logits(self.x_np(), self.W_r.cpu().numpy(), self.bias.cpu().numpy())
+        b = self.bias.cpu().numpy()
+        if self.select_only:
+            z = router.router_logits(self.x_np(), self.W_r.cpu().numpy())
+            return z, router.route(z, self.wl.k, select_bias=b)
+        z = router.router_logits(self.x_np(), self.W_r.cpu().numpy(), b)
         return z, router.route(z, self.wl.k)
 
 

@@ -37,7 +37,13 @@ def test_host_side_argument_checks_without_gpu():
     assert L.moe_plan_create(16, 128, 8, 33, 128, 0, 0, 0, 0, ctypes.byref(h)) == 2
     assert L.moe_plan_create(16, 128, 8, 9, 128, 0, 0, 0, 0, ctypes.byref(h)) == 2
     assert L.moe_plan_create(-1, 128, 8, 2, 128, 0, 0, 0, 0, ctypes.byref(h)) == 1
-    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 1, 0, 0, ctypes.byref(h)) == 1
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 2, 0, 0, ctypes.byref(h)) == 1   # unknown act
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 2, 0, ctypes.byref(h)) == 1   # unknown bias mode
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 0, 1, ctypes.byref(h)) == 1   # unknown flags
+    # both activations and both bias modes are accepted (host-side plan only)
+    for act, mode in ((1, 0), (0, 1), (1, 1)):
+        assert L.moe_plan_create(16, 128, 8, 2, 128, 0, act, mode, 0, ctypes.byref(h)) == 0
+        assert L.moe_plan_destroy(h) == 0
     assert L.moe_quant_mxfp8(None, 4, 33, None, None, None) == 2
     assert L.moe_status_string(3) == b"misaligned pointer"
     sizes = api.moe_expert_bytes(7168, 3072, 896)

@@ -104,8 +104,12 @@ def _check_route(case, atol_z=2e-5):
     z_gpu = logits.cpu().numpy().astype(np.float64)
     z_ref, (idx_o, w_o, gap) = case.oracle_route()
     assert np.max(np.abs(z_gpu - z_ref)) < atol_z
-    # bit-exact selection given identical scores
-    idx_g, w_g, _ = router.route(z_gpu, k)
+    # bit-exact selection given identical scores (select-only: the key z + b in fp32, as
+    # the kernel forms it)
+    if case.select_only:
+        idx_g, w_g, _ = router.route(logits.cpu().numpy(), k, select_bias=case.bias.cpu().numpy())
+    else:
+        idx_g, w_g, _ = router.route(z_gpu, k)
     assert np.array_equal(idx.cpu().numpy(), idx_g)
     assert np.allclose(w.cpu().numpy(), w_g, rtol=2e-6, atol=1e-7)
     # against the oracle's own fp64 routing, mismatches only on near ties
@@ -134,7 +138,7 @@ def _check_layer(case, tokens=None, stage_checks=False):
     y = y.float().cpu().numpy().astype(np.float64)
     x = case.x_np()
     rows = np.arange(case.T) if tokens is None else np.asarray(tokens)
-    y_ref = layer.moe_layer(x, idx_o, w_o, case.oracle_expert, case.oracle_shared(), tokens=rows)
+    y_ref = layer.moe_layer(x, idx_o, w_o, case.oracle_expert, case.oracle_shared(), tokens=rows, act=case.act)
     st = layer_stats(y[rows], y_ref, gap[rows])
     assert st["max_rel"] <= MAX_REL and st["mean_rel"] <= MEAN_REL, st
     if stage_checks:
@@ -172,7 +176,7 @@ def _stage_checks(case, idx, w):
         if len(rows) == 0:
             continue
         Wg, Wu, Wd = case.oracle_expert(e)
-        o_ref, a_ref, hq_ref, hs_ref = layer.expert_forward(X[perm_tok[rows]], Wg, Wu, Wd)
+        o_ref, a_ref, hq_ref, hs_ref = layer.expert_forward(X[perm_tok[rows]], Wg, Wu, Wd, case.act)
         H_ref = mx.dequantize_mx(hq_ref, hs_ref, "e4m3")
         diff = np.abs(H[rows] - H_ref)
         scale = np.repeat(mx.e8m0_value(hs_ref), 32, axis=1)
@@ -235,6 +239,40 @@ def test_layer_tile_configs_agree():
         api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 64)
 
 
+def test_route_select_only_bias():
+    """Select-only bias: logits exclude b, experts are chosen by z + b (fp32), weights from
+    sigmoid(z).  A strong bias makes the chosen set differ from the unbiased top-k."""
+    wl = synth.custom(seed=12, T=300, d=256, E=48, k=6, I=128)
+    bias = torch.zeros(48)
+    bias[torch.randperm(48, generator=torch.Generator().manual_seed(5))[:10]] = 0.5
+    case = Case(wl, bias=bias, select_only=True)
+    idx, w, idx_o, w_o, gap = _check_route(case)
+    z = router.router_logits(case.x_np(), case.W_r.cpu().numpy())
+    plain, _, _ = router.route(z, wl.k)
+    assert not np.array_equal(idx.cpu().numpy(), plain)
+
+
+def test_layer_select_only_bias():
+    wl = synth.custom(seed=13, T=160, d=256, E=16, k=4, I=128, I_shared=128)
+    bias = torch.linspace(-0.5, 0.5, 16)
+    case = Case(wl, bias=bias, select_only=True)
+    _check_layer(case, stage_checks=True)
+
+
+def test_layer_clamped_swiglu():
+    """The clamped SwiGLU on routed and shared experts.  x is scaled by 32 (exact in bf16
+    and MXFP8) so that many pre-activations pass both clamps (|g|, |u| > 7)."""
+    wl = synth.custom(seed=14, T=203, d=384, E=12, k=3, I=256, I_shared=128)
+    case = Case(wl, act="clamped_swiglu", x_scale=32.0)
+    st = _check_layer(case, stage_checks=True)
+    # the clamps are reached: some g of the first expert's rows exceed 7
+    Wg, Wu, _ = case.oracle_expert(0)
+    xq, xs = mx.quantize_mx(case.x_np(), "e4m3")
+    g = mx.dequantize_mx(xq, xs, "e4m3") @ Wg.T
+    assert (g > 7).mean() > 0.01 and (np.abs(mx.dequantize_mx(xq, xs, "e4m3") @ Wu.T) > 7).mean() > 0.01
+    print("clamped", st)
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
@@ -264,3 +302,32 @@ def test_forward_rejects_bad_arguments():
         raw = torch.zeros(4 * 128 + 8, dtype=torch.bfloat16, device="cuda")
         case.plan.forward(raw[1:1 + 512].view(4, 128), idx, w, case.experts)
     assert e.value.code == 3
+
+
+def test_route_and_forward_replay_from_a_cuda_graph():
+    """moe_route + moe_forward make no host synchronisation and allocate nothing, so a
+    whole layer step can be captured into a CUDA graph; replays reproduce the eager bytes."""
+    wl = synth.custom(seed=15, T=96, d=256, E=16, k=4, I=128, I_shared=128)
+    case = Case(wl)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    y = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+
+    def step():
+        api.moe_route(case.plan.handle, case.x, case.W_r, case.bias, wl.k, idx=idx, w=w, stream=s)
+        api.moe_forward(case.plan.handle, case.x, idx, w, case.experts, case.shared, y, stream=s)
+
+    with torch.cuda.stream(s):
+        step()                              # eager run (also sets the kernels' attributes)
+    s.synchronize()
+    y_eager = y.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
+    assert case.plan.check()[0] == 0
