@@ -46,7 +46,7 @@ STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "ga
           "down", "shared_gate_up", "shared_down", "combine"]
 # kernel launches per recorded stage instance (router_gemm: +1 for the partial-sum kernel
 # when moe_plan_get_option(MOE_OPT_ROUTER_SPLIT) > 1)
-STAGE_KERNELS = {"permute": 3}
+STAGE_KERNELS = {"permute": 3, "quant_scatter": 2}
 
 
 class MoeError(RuntimeError):

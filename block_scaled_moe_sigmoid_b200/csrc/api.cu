@@ -133,7 +133,7 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
   size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
-      o_planes, o_xq, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
+      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
   int tokens_per_chunk() const { return kPermThreads; }
   int nchunks(int T) const { return (T + kPermThreads - 1) / kPermThreads; }
   template <class P>
@@ -160,6 +160,7 @@ static void carve(moe_plan_s* p) {
   p->o_xq = take(A * p->d);
   // token-side scale blocks, tile-major: at most A / bn + E group-tiles
   const size_t max_tiles = A / kBNMin + p->E + 1;
+  p->o_xs_tok = take((size_t)p->T_max * (p->d / 32));
   p->o_xs = take(max_tiles * (p->d / 128) * SF_TILE_BYTES);
   p->o_hq = take(A * p->I);
   p->o_hs = take(max_tiles * (p->I / 128) * SF_TILE_BYTES);
@@ -453,9 +454,12 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   {
     const long long n = (long long)T * (d / 32);
     p->prof.begin(MOE_STAGE_QUANT, s);
+    uint8_t* xs_tok = p->at<uint8_t>(p->o_xs_tok);
     quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-        (const uint16_t*)x, T, d, k, idx, p->at<int>(p->o_inv), p->at<int>(p->o_counts),
-        p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), A, xq, xs);
+        (const uint16_t*)x, T, d, k, p->at<int>(p->o_inv), A, xq, xs_tok);
+    const int max_gt = A / bn + E + 1;   // bound on the group-tiles of this call
+    scale_tiles_kernel<<<max_gt, 256, 0, s>>>(xs_tok, d / 32, p->at<int>(p->o_perm), p->at<int>(p->o_counts),
+                                              p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), E, d / 128, xs);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }

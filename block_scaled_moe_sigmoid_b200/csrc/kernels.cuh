@@ -78,57 +78,30 @@ __global__ void quant_mxfp8_kernel(const uint16_t* __restrict__ x, int rows, int
   sc[r * nb + b] = (uint8_t)s;
 }
 
-// Quantise token rows and write each to its k positions in expert order: the elements to
-// xq[inv[t][j]][:], the scales tile-major (tiling.cuh) for the gate/up GEMM.
-// Requires cols % 128 == 0 so four consecutive threads share a row and one scale word.
+// Quantise token rows and write each to its k positions in expert order:
+// xq[inv[t][j]][:] = E4M3 codes of x[t]; the block scales go once per token to
+// xs_tok[t][cols/32] (scale_tiles_kernel turns them into the GEMM's tile-major blocks).
 __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int cols, int k,
-                                     const int* __restrict__ idx, const int* __restrict__ inv,
-                                     const int* __restrict__ counts, const int* __restrict__ offsets,
-                                     const int* __restrict__ tile_prefix, int A_rows,
-                                     uint8_t* __restrict__ xq, uint8_t* __restrict__ xs) {
+                                     const int* __restrict__ inv, int A_rows,
+                                     uint8_t* __restrict__ xq, uint8_t* __restrict__ xs_tok) {
   const int nb = cols >> 5;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool active = gid < (long long)T * nb;
-  const long long t = active ? gid / nb : 0;
-  const int b = active ? (int)(gid - t * nb) : 0;
-  uint4 in[4] = {};
-  if (active) {
-    const uint4* src = (const uint4*)(x + t * cols + b * 32);
+  if (gid >= (long long)T * nb) return;
+  const long long t = gid / nb;
+  const int b = (int)(gid - t * nb);
+  const uint4* src = (const uint4*)(x + t * cols + b * 32);
+  uint4 in[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
-  }
+  for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
   uint32_t out[8];
-  const uint32_t s = quant_block_e4m3(in, out);
-  // gather the 4 scale bytes of blocks 4m..4m+3 into lane 4m's word
-  const int l = threadIdx.x & 31;
-  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
-  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
-  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
-  if (!active) return;
-  const uint32_t word = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  xs_tok[gid] = (uint8_t)quant_block_e4m3(in, out);
   const uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
   const uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
-  const int k_tiles = cols >> 7;
-  const bool sc_lane = (l & 3) == 0;   // this lane writes the 4-block scale word
-  // four destinations at a time, so that their index loads and tile lookups overlap
+  // four destinations at a time, so that their index loads overlap
   for (int j0 = 0; j0 < k; j0 += 4) {
-    int pj[4], ej[4];
+    int pj[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = j0 + q;
-      pj[q] = j < k ? __ldg(inv + t * k + j) : -1;
-      ej[q] = (j < k && sc_lane) ? __ldg(idx + t * k + j) : 0;
-    }
-    size_t soff[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      soff[q] = 0;
-      if (sc_lane && pj[q] >= 0 && pj[q] < A_rows) {
-        int gt, n;
-        row_tile(counts, offsets, tile_prefix, ej[q], pj[q], gt, n);
-        soff[q] = ((size_t)gt * k_tiles + (b >> 2)) * SF_TILE_BYTES + sf_atom_offset(n);
-      }
-    }
+    for (int q = 0; q < 4; ++q) pj[q] = j0 + q < k ? __ldg(inv + t * k + j0 + q) : -1;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int p = pj[q];
@@ -136,8 +109,41 @@ __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int 
       uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
       dst[0] = o0;
       dst[1] = o1;
-      if (sc_lane) *(uint32_t*)(xs + soff[q]) = word;
     }
+  }
+}
+
+// Token-side scale blocks of the gate/up GEMM, tile-major (tiling.cuh): one CTA per
+// group-tile, one thread per row of the tile's scale atoms.  Row n of group-tile gt takes
+// the four block scales of K tile kt of its token, xs_tok[perm_tok[row0 + n]][4 kt ..],
+// as one word; rows past the tile's valid rows get zero scales.  Each CTA writes its
+// k_tiles blocks whole, so no partial sectors reach DRAM.
+__global__ void __launch_bounds__(256)
+    scale_tiles_kernel(const uint8_t* __restrict__ xs_tok, int nb, const int* __restrict__ perm_tok,
+                       const int* __restrict__ counts, const int* __restrict__ offsets,
+                       const int* __restrict__ tile_prefix, int E, int k_tiles, uint8_t* __restrict__ xs) {
+  const int gt = blockIdx.x;
+  if (gt >= __ldg(tile_prefix + E)) return;
+  int lo = 0, hi = E - 1;   // last group whose first tile is <= gt
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(tile_prefix + mid) <= gt) lo = mid; else hi = mid - 1;
+  }
+  const int tp = __ldg(tile_prefix + lo);
+  const int ntiles = __ldg(tile_prefix + lo + 1) - tp;
+  const int rows = __ldg(counts + lo);
+  const int n_per = tile_rows_per(rows, ntiles);
+  const int nt = gt - tp;
+  const int n_valid = min(n_per, rows - nt * n_per);
+  const int atoms = (((n_valid + 15) & ~15) + 127) >> 7;
+  const int n = threadIdx.x;
+  if (n >= atoms * 128) return;
+  const bool valid = n < n_valid;
+  const uint8_t* src = xs_tok + (valid ? (size_t)__ldg(perm_tok + __ldg(offsets + lo) + nt * n_per + n) * nb : 0);
+  uint8_t* dst = xs + (size_t)gt * k_tiles * SF_TILE_BYTES + sf_atom_offset(n);
+  for (int kt = 0; kt < k_tiles; ++kt) {
+    const uint32_t v = valid ? __ldg((const uint32_t*)(src + kt * 4)) : 0u;
+    *(uint32_t*)(dst + (size_t)kt * SF_TILE_BYTES) = v;
   }
 }
 

@@ -81,6 +81,10 @@ WORKLOADS = {
     # Kimi-K3 expert shapes on a 64-expert slice (2.2 GB of weights): a profiling case that
     # keeps the device footprint to a few GB while the weights still exceed L2
     "k3_slice_e64_t1024": Workload("k3_slice_e64_t1024", 2, 1024, 7168, 64, 16, 3072, 3072, device="cuda"),
+    # the pages' shared expert: two full-width experts stored fused as one GLU with
+    # intermediate size 6144 ("Kimi K3.1 Pro vs gpt-oss-120b", component table, shared-expert row)
+    "k3_prefill_t8192_shared6144": Workload("k3_prefill_t8192_shared6144", 2, 8192, 7168, 896, 16, 3072, 6144,
+                                            device="cuda"),
     # token-count sweep (T is given per run)
     "k3_sweep": Workload("k3_sweep", 4, 1, 7168, 896, 16, 3072, 3072, device="cuda",
                          sweep=(1, 16, 256, 2048, 16384)),

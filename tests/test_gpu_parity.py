@@ -273,6 +273,14 @@ def test_layer_clamped_swiglu():
     print("clamped", st)
 
 
+def test_layer_fused_double_shared_expert():
+    """The pages' shared expert is two full-width experts fused into one GLU of twice the
+    intermediate size; here I_shared = 2 I."""
+    wl = synth.custom(seed=16, T=130, d=256, E=8, k=2, I=128, I_shared=256)
+    case = Case(wl)
+    _check_layer(case, stage_checks=True)
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
