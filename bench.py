@@ -31,7 +31,7 @@ UNIT = "tokens/s"
 # workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` of this
 # kernel version (profiles/dram_gemm_k3_prefill_t8192.md).  None whenever the kernel
 # has changed since that capture.
-GATE_UP_TRAFFIC_BYTES = {8192: 24134107648 + 412293120}
+GATE_UP_TRAFFIC_BYTES = {}
 
 
 def parse():
@@ -154,6 +154,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+def max_over_ranks_(v, world, device):
+    """The largest of the ranks' values (every rank gets it); v itself when world == 1."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(T, steps, world, ms_max):
+    """Whole-job tokens/s: every rank runs `steps` steps of T tokens; the job takes the
+    slowest rank's time."""
+    return world * T * steps / (ms_max / 1e3)
+
+
 # ---------------------------------------------------------------- our arm
 def setup(wl, T, device):
     import torch
@@ -206,11 +224,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
+        return max_over_ranks_(v, world, dev)
 
     # ---- timed region (device time, CUDA events on the launching stream)
     clocks = ClockSampler(local_rank)
@@ -313,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
 
     out = None
     if rank == 0:
-        value = world * T * args.steps / (ms / 1e3)
+        value = job_throughput(T, args.steps, world, ms)
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,

@@ -30,7 +30,7 @@ Readings (the pages leave these open):
       rounded to bf16 (the precision of the operand of the second product).
   R16 Output: y = y_shared + sum_j w_j * o_j accumulated in fp64, then rounded
       once to bf16 (ties to even).
-  R17 Second GLU (an option, not the Kimi default): the clamped SwiGLU that
+  R21 Second GLU (an option, not the Kimi default): the clamped SwiGLU that
       "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, routed-experts
       row, describes for gpt-oss.  The gate is clamped from above at 7.0, the
       linear branch to [-7, 7], and a = (u_c + 1) * g_c * sigmoid(1.702 g_c).
@@ -53,7 +53,7 @@ def glu_silu(g, u):
 
 
 def glu_clamped_swiglu(g, u, limit=7.0, alpha=1.702):
-    """Clamped SwiGLU (R17): (clip(u, -7, 7) + 1) * g_c * sigmoid(1.702 g_c), g_c = min(g, 7)."""
+    """Clamped SwiGLU (R21): (clip(u, -7, 7) + 1) * g_c * sigmoid(1.702 g_c), g_c = min(g, 7)."""
     gc = np.minimum(np.asarray(g, dtype=np.float64), limit)
     uc = np.clip(np.asarray(u, dtype=np.float64), -limit, limit)
     return (uc + 1.0) * gc / (1.0 + np.exp(-alpha * gc))
@@ -83,7 +83,7 @@ def decode_expert(q):
 
 
 def expert_hidden(X, Wg, Wu, act="silu"):
-    """a = glu(X Wg^T, X Wu^T) in fp64 (R11, R13, R17).  X: [M, d] exact values."""
+    """a = glu(X Wg^T, X Wu^T) in fp64 (R11, R13, R21).  X: [M, d] exact values."""
     g = X @ Wg.T
     u = X @ Wu.T
     return ACTIVATIONS[act](g, u)

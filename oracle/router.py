@@ -20,7 +20,7 @@ Readings (the pages leave these open):
      The output order is the selection order.
   R9 The "16th/17th gap" of a token is sigmoid(z_(k)) - sigmoid(z_(k+1)) in fp64
      (z_(i) is the i-th largest logit); it is +inf when k == E.
-  R10 Select-only bias (second mode).  The same rows call b a per-expert
+  R20 Select-only bias (second mode).  The same rows call b a per-expert
      *selection* bias, and the raw config of "Kimi K3" (llm-atlas) has
      topk_method noaux_tc.  The plainest reading of both: experts are chosen
      by z + b, while the weights come from the unbiased s = sigmoid(z).  Ties
@@ -70,7 +70,7 @@ def route(z, k, select_bias=None):
     """Selection, renormalised weights and the k/k+1 score gap (R7, R8, R9).
 
     select_bias: None (any bias is already inside z, R6) or the [E] bias of the
-    select-only mode (R10): selection by z + b, weights from sigmoid(z).
+    select-only mode (R20): selection by z + b, weights from sigmoid(z).
     Returns (idx int32 [T,k], w fp64 [T,k], gap fp64 [T]).
     """
     z_in = np.asarray(z)

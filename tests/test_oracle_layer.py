@@ -177,7 +177,7 @@ def test_relative_error_definition():
     assert abs(nw[0] - math.sqrt(0.01 ** 2 + 0.001 ** 2) / math.sqrt(5.25)) < 1e-15
 
 
-# ------------------------------------------------------------------ clamped SwiGLU (R17)
+# ------------------------------------------------------------------ clamped SwiGLU (R21)
 def test_clamped_swiglu_inside_the_clamps_is_scaled_torch_silu():
     """Inside the clamps, (u + 1) * g * sigmoid(1.702 g) equals (u + 1) * silu(1.702 g) / 1.702.
     torch's silu (a library routine) pins the sigmoid factor and which operand is the gate."""

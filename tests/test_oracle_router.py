@@ -114,7 +114,7 @@ def test_config_closed_forms():
     assert int(cfg["hidden_size"]) == 2 * dl
 
 
-# ------------------------------------------------------------------ select-only bias (R10)
+# ------------------------------------------------------------------ select-only bias (R20)
 def test_select_only_bias_brute_force():
     """Selection by z + b (full sort, lower index on ties), weights from sigmoid(z)."""
     rng = np.random.default_rng(21)
