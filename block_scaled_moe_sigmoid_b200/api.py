@@ -266,16 +266,17 @@ class Shared:
 
 MOE_ACT_SILU_GLU, MOE_ACT_CLAMPED_SWIGLU = 0, 1
 MOE_BIAS_LOGIT, MOE_BIAS_SELECT_ONLY = 0, 1
+MOE_FLAG_STATIC_ROUTER = 1
 
 
 class Plan:
     """A plan plus its torch-allocated workspace."""
 
     def __init__(self, T_max, d, E, k, I, I_shared=0, device="cuda", act=MOE_ACT_SILU_GLU,
-                 bias_mode=MOE_BIAS_LOGIT):
+                 bias_mode=MOE_BIAS_LOGIT, flags=0):
         self.T_max, self.d, self.E, self.k, self.I, self.I_shared = T_max, d, E, k, I, I_shared
-        self.act, self.bias_mode = act, bias_mode
-        self.handle = moe_plan_create(T_max, d, E, k, I, I_shared, act, bias_mode)
+        self.act, self.bias_mode, self.flags = act, bias_mode, flags
+        self.handle = moe_plan_create(T_max, d, E, k, I, I_shared, act, bias_mode, flags)
         n = moe_plan_workspace_bytes(self.handle)
         self.workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
         moe_plan_set_workspace(self.handle, self.workspace)

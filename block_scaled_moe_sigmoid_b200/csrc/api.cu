@@ -120,6 +120,8 @@ struct moe_plan_s {
   int pf_dist = 0, pf_b = 0;  // GEMM L2 prefetch (moe_plan_set_option)
   int act = MOE_ACT_SILU_GLU;
   int bias_mode = MOE_BIAS_LOGIT;
+  int flags = 0;
+  const void* planes_of = nullptr;   // W_r the router planes were last split from
   int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
   int last_bn = 0;            // token rows per tile in the last moe_forward
   int last_ksplit = 0;        // router K splits in the last moe_route
@@ -249,7 +251,7 @@ moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared
   if (!out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   if ((act != MOE_ACT_SILU_GLU && act != MOE_ACT_CLAMPED_SWIGLU) ||
-      (bias_mode != MOE_BIAS_LOGIT && bias_mode != MOE_BIAS_SELECT_ONLY) || flags != 0)
+      (bias_mode != MOE_BIAS_LOGIT && bias_mode != MOE_BIAS_SELECT_ONLY) || (flags & ~MOE_FLAG_STATIC_ROUTER))
     return MOE_ERR_INVALID_ARG;
   if (T_max < 0 || d <= 0 || E <= 0 || k <= 0 || I <= 0 || I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (d % 128 || I % 128 || I_shared % 128 || k > E || k > 32 || E > 4096)
@@ -259,6 +261,7 @@ moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared
   p->T_max = T_max; p->d = d; p->E = E; p->k = k; p->I = I; p->Is = I_shared;
   p->act = act;
   p->bias_mode = bias_mode;
+  p->flags = flags;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) {
     int sms = 0;
@@ -282,6 +285,7 @@ moe_status_t moe_plan_set_workspace(moe_plan_t p, void* dev_ptr, size_t bytes) {
   if (bytes < p->total) return MOE_ERR_INVALID_ARG;
   p->ws = (char*)dev_ptr;
   p->ws_bytes = bytes;
+  p->planes_of = nullptr;   // the router planes live in the workspace
   if (cudaMemset(p->ws + p->o_status, 0, 256) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
@@ -355,9 +359,12 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   __nv_bfloat16* planes = p->at<__nv_bfloat16>(p->o_planes);
   float* z = logits_opt ? logits_opt : p->at<float>(p->o_logits);
   if (!aligned(z, 16)) return MOE_ERR_ALIGNMENT;
-  p->prof.begin(MOE_STAGE_ROUTER_SPLIT, s);
-  router_split_kernel<<<dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s>>>(W_r, d, E, planes);
-  p->prof.end(s);
+  if (!(p->flags & MOE_FLAG_STATIC_ROUTER) || p->planes_of != (const void*)W_r) {
+    p->prof.begin(MOE_STAGE_ROUTER_SPLIT, s);
+    router_split_kernel<<<dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s>>>(W_r, d, E, planes);
+    p->prof.end(s);
+    p->planes_of = W_r;
+  }
   CUtensorMap tA, tB;
   if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, planes, 3ull * d, E, 3ull * d * 2, 64, 128) ||
       !make_map(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, (uint64_t)d * 2, 64, 32))

@@ -98,7 +98,13 @@ typedef struct {
  * moe_plan_create: checks the layer shape and the device, allocates nothing on the
  * device.  T_max bounds the tokens of any later call; d, I, I_shared multiples of 128
  * (I_shared = 0: no shared expert); 1 <= k <= min(E, 32); E <= 4096.
+ * flags: 0 or MOE_FLAG_STATIC_ROUTER.  With it, moe_route splits W_r into its three bf16
+ * terms only when W_r is a different pointer from the one it split last (or on the first
+ * call) and reuses them otherwise.  The caller then must not change the contents behind
+ * an unchanged pointer; inference weights qualify.  Without it, every call splits again
+ * (E*d*4 bytes in, E*d*6 out).  Any other bit is MOE_ERR_INVALID_ARG.
  * Returns the plan in *out (host object, freed by moe_plan_destroy). */
+enum { MOE_FLAG_STATIC_ROUTER = 1 };
 moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared,
                              moe_act_t act, moe_bias_mode_t bias_mode, int flags,
                              moe_plan_t* out);

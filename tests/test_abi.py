@@ -39,7 +39,9 @@ def test_host_side_argument_checks_without_gpu():
     assert L.moe_plan_create(-1, 128, 8, 2, 128, 0, 0, 0, 0, ctypes.byref(h)) == 1
     assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 2, 0, 0, ctypes.byref(h)) == 1   # unknown act
     assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 2, 0, ctypes.byref(h)) == 1   # unknown bias mode
-    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 0, 1, ctypes.byref(h)) == 1   # unknown flags
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 0, 2, ctypes.byref(h)) == 1   # unknown flag bit
+    assert L.moe_plan_create(16, 128, 8, 2, 128, 0, 0, 0, 1, ctypes.byref(h)) == 0   # static router
+    assert L.moe_plan_destroy(h) == 0
     # both activations and both bias modes are accepted (host-side plan only)
     for act, mode in ((1, 0), (0, 1), (1, 1)):
         assert L.moe_plan_create(16, 128, 8, 2, 128, 0, act, mode, 0, ctypes.byref(h)) == 0

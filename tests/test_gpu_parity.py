@@ -281,6 +281,26 @@ def test_layer_fused_double_shared_expert():
     _check_layer(case, stage_checks=True)
 
 
+def test_static_router_flag_reuses_and_refreshes_planes():
+    """MOE_FLAG_STATIC_ROUTER: the second call with the same W_r skips the split and gives
+    the same logits; a call with another W_r pointer splits that matrix."""
+    wl = synth.custom(seed=17, T=64, d=256, E=24, k=4, I=128)
+    case = Case(wl)
+    plan = api.Plan(wl.T, wl.d, wl.E, wl.k, wl.I, flags=api.MOE_FLAG_STATIC_ROUTER)
+    z0 = torch.empty((wl.T, wl.E), device="cuda")
+    z1 = torch.empty_like(z0)
+    i0, w0 = plan.route(case.x, case.W_r, case.bias, logits=z0)
+    i1, w1 = plan.route(case.x, case.W_r, case.bias, logits=z1)
+    assert torch.equal(z0, z1) and torch.equal(i0, i1) and torch.equal(w0, w1)
+    W2 = (case.W_r * 2.0).contiguous()          # exact scaling: logits double exactly
+    z2 = torch.empty_like(z0)
+    plan.route(case.x, W2, None, logits=z2)
+    zb = torch.empty_like(z0)
+    plan.route(case.x, case.W_r, None, logits=zb)
+    assert torch.equal(z2, 2.0 * zb)
+    assert plan.check()[0] == 0
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
