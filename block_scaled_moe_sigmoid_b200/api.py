@@ -35,6 +35,7 @@ SIGNATURES = {
     "moe_pack_expert_mxfp4": [_I, _I, _I, _P, _P, _P, _P, _P],
     "moe_pack_shared_bf16": [_I, _I, _P, _P, _P, _P, _P],
     "moe_debug_buffer": [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_S)],
+    "moe_debug_timeout_probe": [_P, _P],
     "moe_plan_set_profiling": [_P, _I],
     "moe_plan_set_option": [_P, _I, _I],
     "moe_plan_get_option": [_P, _I, ctypes.POINTER(_I)],
@@ -118,6 +119,11 @@ def moe_plan_check(plan, stream=None):
     bits = ctypes.c_uint()
     code = lib().moe_plan_check(plan, _stream(stream), ctypes.byref(bits))
     return code, bits.value
+
+
+def moe_debug_timeout_probe(plan, stream=None):
+    """One bounded wait that runs out on the GPU (see include/moe.h)."""
+    _call("moe_debug_timeout_probe", plan, _stream(stream))
 
 
 def moe_plan_destroy(plan):

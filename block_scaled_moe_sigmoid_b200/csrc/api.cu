@@ -202,7 +202,6 @@ static GemmArgs base_args(const moe_plan_s* p) {
   a.dense_rows = -1;
   a.pf_dist = p->pf_dist;
   a.pf_b = p->pf_b;
-  a.act = p->act;
   return a;
 }
 
@@ -498,7 +497,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.out1 = hs;
     a.ld_out = I;
     p->prof.begin(MOE_STAGE_GATE_UP, s);
-    if (launch_gemm<KIND_MX, EPI_GLU_MX8>(bn, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
+        ? launch_gemm<KIND_MX, EPI_GLU_MX8_CLAMPED>(bn, a, tA, tB, p->num_sms, s)
+        : launch_gemm<KIND_MX, EPI_GLU_MX8>(bn, a, tA, tB, p->num_sms, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
   // a7: down grouped GEMM -> O (bf16, expert order)
@@ -550,7 +552,10 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.ld_out = Is;
     int tiles = ((T + bn - 1) / bn) * a.m_tiles;
     p->prof.begin(MOE_STAGE_SHARED_GATE_UP, s);
-    if (launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s) != cudaSuccess)
+    const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
+        ? launch_gemm<KIND_BF16, EPI_GLU_BF16_CLAMPED>(bn, a, tA, tB, std::min(tiles, p->num_sms), s)
+        : launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s);
+    if (e != cudaSuccess)
       return MOE_ERR_CUDA;
     p->prof.end(s);
     CUtensorMap tA2;
@@ -689,6 +694,13 @@ moe_status_t moe_plan_stage_ms(moe_plan_t p, float* ms, int* launches, int n) {
   p->prof.recs.clear();
   p->prof.used = 0;
   return MOE_OK;
+}
+
+moe_status_t moe_debug_timeout_probe(moe_plan_t p, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  timeout_probe_kernel<<<1, 32, 0, S(stream)>>>(p->at<unsigned int>(p->o_status));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes) {

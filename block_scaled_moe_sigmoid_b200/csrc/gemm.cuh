@@ -34,10 +34,19 @@ namespace moe {
 
 enum { KIND_MX = 0, KIND_BF16 = 1 };
 enum {
-  EPI_GLU_MX8 = 0,   // a = glu(gate, up), requantised to MXFP8 along the channels
-  EPI_GLU_BF16 = 1,  // a = glu(gate, up), stored as bf16
-  EPI_BF16 = 2,      // D stored as bf16
-  EPI_F32 = 3        // D stored as fp32
+  EPI_GLU_MX8 = 0,          // a = silu(gate) * up, requantised to MXFP8 along the channels
+  EPI_GLU_BF16 = 1,         // a = silu(gate) * up, stored as bf16
+  EPI_BF16 = 2,             // D stored as bf16
+  EPI_F32 = 3,              // D stored as fp32
+  EPI_GLU_MX8_CLAMPED = 4,  // as EPI_GLU_MX8 with the clamped SwiGLU (glu_f<1>)
+  EPI_GLU_BF16_CLAMPED = 5  // as EPI_GLU_BF16 with the clamped SwiGLU
+};
+template <int EPI>
+struct EpiTraits {
+  static constexpr bool glu = EPI == EPI_GLU_MX8 || EPI == EPI_GLU_BF16 || EPI == EPI_GLU_MX8_CLAMPED ||
+                              EPI == EPI_GLU_BF16_CLAMPED;
+  static constexpr bool mx8_out = EPI == EPI_GLU_MX8 || EPI == EPI_GLU_MX8_CLAMPED;
+  static constexpr int act = (EPI == EPI_GLU_MX8_CLAMPED || EPI == EPI_GLU_BF16_CLAMPED) ? 1 : 0;
 };
 
 struct GemmArgs {
@@ -60,7 +69,6 @@ struct GemmArgs {
   int pf_dist;          // L2 prefetch distance in k-tiles (0 = off), KIND_MX weights
   int pf_b;             // reserved
   const uint8_t* a_ptr; // KIND_MX: packed weights (base of the tile-major code array)
-  int act;              // GLU epilogues: MOE_ACT_SILU_GLU (0) or MOE_ACT_CLAMPED_SWIGLU (1)
 };
 
 template <int KIND, int BN_MAX, int STAGES>
@@ -128,13 +136,17 @@ __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, 
 }
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
-// a = glu(g, u): act 0 SiLU-GLU; act 1 clamped SwiGLU, (clamp(u, -7, 7) + 1) * g_c *
+// a = glu(g, u): ACT 0 SiLU-GLU; ACT 1 clamped SwiGLU, (clamp(u, -7, 7) + 1) * g_c *
 // sigmoid(1.702 g_c) with g_c = min(g, 7)
-__device__ __forceinline__ float glu_f(int act, float g, float u) {
-  if (act == 0) return silu_f(g) * u;
-  const float gc = fminf(g, 7.0f);
-  const float uc = fminf(fmaxf(u, -7.0f), 7.0f);
-  return (uc + 1.0f) * __fdividef(gc, 1.0f + __expf(-1.702f * gc));
+template <int ACT>
+__device__ __forceinline__ float glu_f(float g, float u) {
+  if constexpr (ACT == 0) {
+    return silu_f(g) * u;
+  } else {
+    const float gc = fminf(g, 7.0f);
+    const float uc = fminf(fmaxf(u, -7.0f), 7.0f);
+    return (uc + 1.0f) * __fdividef(gc, 1.0f + __expf(-1.702f * gc));
+  }
 }
 
 // MXFP8 (E4M3) encoding of v with block scale exponent from the block's amax bits.
@@ -436,7 +448,7 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(acc_empty));
       };
-      if constexpr (EPI == EPI_GLU_MX8 || EPI == EPI_GLU_BF16) {
+      if constexpr (EpiTraits<EPI>::glu) {
         // a = glu(g, u) for this warp's chunks (c = sub + 2 i) straight out of TMEM;
         // TMEM goes back to the MMA warp before the quantisation and stores.
         float a[CH / 2][16];
@@ -449,7 +461,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld16(lane_base + BN_MAX + c * 16, u);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a[i][j] = glu_f(args.act, __uint_as_float(g[j]), __uint_as_float(u[j]));
+            for (int j = 0; j < 16; ++j) a[i][j] = glu_f<EpiTraits<EPI>::act>(__uint_as_float(g[j]), __uint_as_float(u[j]));
           }
         }
         release_tmem();
@@ -463,7 +475,7 @@ __global__ void __launch_bounds__(384, 1)
             const int n = c * 16 + j;
             if (n >= ti.n_valid) break;
             const size_t row = (size_t)(ti.row0 + n);
-            if constexpr (EPI == EPI_GLU_MX8) {
+            if constexpr (EpiTraits<EPI>::mx8_out) {
               const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a[i][j]) & 0x7FFFFFFFu);
               const int e = mx_exp_e4m3(amax);
               const float qv = a[i][j] * __uint_as_float((uint32_t)(127 - e) << 23);

@@ -404,6 +404,22 @@ __global__ void __launch_bounds__(kCombineThreads)
   *(uint4*)(y + (size_t)t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// ---------------------------------------------------------------- failure-path probe
+// One thread waits on an mbarrier of count 1 that nothing arrives at, with the bounded
+// wait of the production kernels; it gives up after the limit and flags the status word.
+__global__ void timeout_probe_kernel(unsigned int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, status, (volatile int*)&abort_flag);
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- weight packing (setup)
 // fp32 rows [R][K] -> E2M1 codes (2 per byte, element 2j in the low nibble) for packed row
 // dst_row(r) in the tile-major code layout [m-tile][K/128][256 rows][64 B], and E8M0

@@ -253,6 +253,15 @@ moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n)
  * Row counts use the T of the last call. */
 moe_status_t moe_debug_buffer(moe_plan_t plan, int which, void** dev_ptr, size_t* bytes);
 
+/* ---- failure-path probe -----------------------------------------------------------------
+ * Launches one CTA on `stream` that waits, with the same bounded mbarrier wait the GEMM
+ * and router kernels use, on a barrier that nothing ever arrives at.  After the wait's
+ * limit (1 s of %globaltimer) the kernel records MOE_ERR_TIMEOUT in the plan's status word
+ * and returns.  The context stays usable, and the next moe_plan_check reports
+ * MOE_ERR_TIMEOUT and clears it.  It tests the timeout path without faulting or hanging
+ * the GPU.  Needs the plan's workspace. */
+moe_status_t moe_debug_timeout_probe(moe_plan_t plan, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

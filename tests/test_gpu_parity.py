@@ -301,6 +301,13 @@ def test_static_router_flag_reuses_and_refreshes_planes():
     assert plan.check()[0] == 0
 
 
+def test_layer_max_top_k_32():
+    """The largest supported k (32) with more experts than one 128-lane router tile."""
+    wl = synth.custom(seed=18, T=40, d=256, E=160, k=32, I=128, I_shared=128)
+    case = Case(wl)
+    _check_layer(case, stage_checks=True)
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
