@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <atomic>
 #include <vector>
 
 #include "../../include/moe.h"
@@ -172,17 +173,27 @@ static void carve(moe_plan_s* p) {
   p->total = o;
 }
 
+// cudaFuncSetAttribute acts on the current device: remember, per kernel and per device
+// (bit d of `done`), which ones already had their dynamic shared-memory limit raised.
+template <class K>
+static cudaError_t ensure_smem_attr(K kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 template <int KIND, int EPI, int BN, int STAGES>
 static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
                                    cudaStream_t s) {
   using Cfg = GemmCfg<KIND, BN, STAGES>;
   auto kern = gemm_kernel<KIND, EPI, BN, STAGES>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  const cudaError_t e = ensure_smem_attr(kern, Cfg::SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s>>>(a, tA, tB);
   return cudaGetLastError();
@@ -206,13 +217,10 @@ static GemmArgs base_args(const moe_plan_s* p) {
 }
 
 static cudaError_t set_smem_attrs() {
-  static cudaError_t st = [] {
-    cudaError_t e = cudaFuncSetAttribute(perm_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topk_sigmoid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    return e;
-  }();
-  return st;
+  static std::atomic<uint64_t> place_done{0}, topk_done{0};
+  cudaError_t e = ensure_smem_attr(perm_place_kernel, 160 * 1024, place_done);
+  if (e == cudaSuccess) e = ensure_smem_attr(topk_sigmoid_kernel, 160 * 1024, topk_done);
+  return e;
 }
 
 // histogram -> scan -> placement into the plan workspace
@@ -407,8 +415,8 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
-    static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, RC::SMEM_BYTES);
-    if (attr != cudaSuccess) return MOE_ERR_CUDA;
+    static std::atomic<uint64_t> router_done{0};
+    if (ensure_smem_attr(kern, RC::SMEM_BYTES, router_done) != cudaSuccess) return MOE_ERR_CUDA;
     const int tiles = base_tiles * ra.ksplit;
     p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
     kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);

@@ -36,6 +36,17 @@ Readings (the pages leave these open):
       linear branch to [-7, 7], and a = (u_c + 1) * g_c * sigmoid(1.702 g_c).
       Reading: "gate" is the first projection g and "linear branch" the second u.
       The plan's activation applies to every GLU of the layer, routed and shared.
+  R22 Latent option (not the default; unpinned placement).  The component tables of
+      "Kimi K3.1 Pro vs gpt-oss-120b" and "Gemma 4 31B vs Kimi K3" have the routed
+      experts run in a 3,584-dim latent (half of d) with an RMSNorm before the
+      up-projection.  The raw config of "Kimi K3" (llm-atlas) gives
+      routed_expert_hidden_size 3584, latent_moe_use_norm true and rms_norm_eps 1e-5.
+      The projections' placement, weights and precision are not published.  Plainest
+      reading, built as an option:
+        x_l = x W_ld^T (bf16 weights, fp32/fp64 accumulation)
+        x_n = bf16(x_l / sqrt(mean(x_l^2) + eps) * gamma)   (the norm before the experts' up-projection)
+        y_l = bf16(sum_j w_j expert_j(x_n))                  (experts act on the latent)
+        y   = bf16(y_l W_lu^T + shared(x))                   (the shared expert reads the un-projected x)
 """
 import numpy as np
 
@@ -161,6 +172,36 @@ def moe_layer(x, idx, w, expert_weights, shared=None, tokens=None, act="silu",
         inter["xq"], inter["xs"] = xq, xs
         return y, inter
     return y
+
+
+def rms_norm(v, gamma, eps=1e-5):
+    """v / sqrt(mean(v^2) + eps) * gamma over the last axis, in fp64 (R22)."""
+    v = np.asarray(v, dtype=np.float64)
+    ms = np.mean(v * v, axis=-1, keepdims=True)
+    return v / np.sqrt(ms + eps) * np.asarray(gamma, dtype=np.float64)
+
+
+def latent_moe_layer(x, idx, w, expert_weights, latent, shared=None, tokens=None, act="silu",
+                     eps=1e-5):
+    """The latent option (R22) for the rows `tokens` of x.
+
+    latent: (W_ld [dl, d] bf16 values, gamma [dl], W_lu [d, dl] bf16 values);
+    expert_weights(e) -> decoded expert weights acting on the dl-dim latent.
+    Returns y fp64 [len(tokens), d] holding bf16 values.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    W_ld, gamma, W_lu = (np.asarray(a, dtype=np.float64) for a in latent)
+    T = x.shape[0]
+    rows = np.arange(T) if tokens is None else np.asarray(tokens)
+    xn = np.zeros((T, W_ld.shape[0]))
+    xn[rows] = mx.bf16_round(rms_norm(x[rows] @ W_ld.T, gamma, eps))
+    y_l = moe_layer(xn, idx, w, expert_weights, None, tokens=rows, act=act)   # bf16(sum_j w_j o_j)
+    y_r = y_l @ W_lu.T
+    if shared is not None:
+        ys, _ = shared_expert(x[rows], *shared, act=act)
+    else:
+        ys = np.zeros_like(y_r)
+    return mx.bf16_round(y_r + ys)
 
 
 def relative_errors(y, y_ref):

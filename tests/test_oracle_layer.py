@@ -221,3 +221,60 @@ def test_single_expert_clamped_swiglu_torch():
     hq, hs = mx.quantize_mx(a.numpy(), "e4m3")
     o = F.linear(torch.from_numpy(mx.dequantize_mx(hq, hs, "e4m3")), Wd).numpy()
     assert np.allclose(y, mx.bf16_round(o), rtol=2 ** -7, atol=0)
+
+
+# ------------------------------------------------------------------ latent option (R22)
+def test_rms_norm_matches_torch():
+    rng = np.random.default_rng(31)
+    v = rng.standard_normal((9, 96)) * rng.uniform(0.01, 30.0, (9, 1))
+    gamma = rng.uniform(0.5, 1.5, 96)
+    ref = F.rms_norm(torch.from_numpy(v), (96,), torch.from_numpy(gamma), eps=1e-5).numpy()
+    assert np.allclose(layer.rms_norm(v, gamma), ref, rtol=1e-13, atol=0)
+
+
+def test_latent_single_expert_is_dense_pipeline_torch():
+    """E = k = 1 in the latent option: x -> W_ld -> RMSNorm -> bf16 -> one quantised GLU MLP
+    -> bf16 -> W_lu, plus the shared expert, all through torch float64 linears."""
+    rng = np.random.default_rng(32)
+    T, d, dl, I = 12, 128, 64, 32
+    x = _bf16(rng.standard_normal((T, d)))
+    W_ld = _bf16(rng.standard_normal((dl, d)) * 0.05)
+    W_lu = _bf16(rng.standard_normal((d, dl)) * 0.05)
+    gamma = rng.uniform(0.5, 1.5, dl)
+    Ws = _experts(rng, 1, dl, I)
+    shared = tuple(_bf16(rng.standard_normal(sh) * 0.02) for sh in ((48, d), (48, d), (d, 48)))
+    idx = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1))
+    y = layer.latent_moe_layer(x, idx, w, lambda e: Ws[0], (W_ld, gamma, W_lu), shared)
+
+    xt = torch.from_numpy(x)
+    xl = F.linear(xt, torch.from_numpy(W_ld))
+    xn = F.rms_norm(xl, (dl,), torch.from_numpy(gamma), eps=1e-5).to(torch.bfloat16).to(torch.float64)
+    xq, xs = mx.quantize_mx(xn.numpy(), "e4m3")
+    X = torch.from_numpy(mx.dequantize_mx(xq, xs, "e4m3"))
+    Wg, Wu, Wd = (torch.from_numpy(a) for a in Ws[0])
+    a = F.silu(F.linear(X, Wg)) * F.linear(X, Wu)
+    hq, hs = mx.quantize_mx(a.numpy(), "e4m3")
+    o = F.linear(torch.from_numpy(mx.dequantize_mx(hq, hs, "e4m3")), Wd)
+    yl = o.to(torch.bfloat16).to(torch.float64)
+    yr = F.linear(yl, torch.from_numpy(W_lu))
+    ys, _ = layer.shared_expert(x, *shared)
+    ref = mx.bf16_round(yr.numpy() + ys)
+    # torch's rms_norm and the bf16 casts may round a few elements differently from fp64
+    assert np.mean(y == ref) > 0.98
+    assert np.allclose(y, ref, rtol=2 ** -6, atol=1e-6)
+
+
+def test_latent_routing_slices_and_token_subset():
+    """Rows of a token subset equal the same rows of the full computation."""
+    rng = np.random.default_rng(33)
+    T, d, dl, I, E, k = 20, 128, 64, 32, 4, 2
+    x = _bf16(rng.standard_normal((T, d)))
+    lat = (_bf16(rng.standard_normal((dl, d)) * 0.05), rng.uniform(0.5, 1.5, dl),
+           _bf16(rng.standard_normal((d, dl)) * 0.05))
+    Ws = _experts(rng, E, dl, I)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = rng.uniform(0.1, 1.0, (T, k))
+    full = layer.latent_moe_layer(x, idx, w, lambda e: Ws[e], lat)
+    rows = np.array([3, 7, 19])
+    assert np.array_equal(layer.latent_moe_layer(x, idx, w, lambda e: Ws[e], lat, tokens=rows), full[rows])
