@@ -81,15 +81,30 @@ def oracle_sample_seconds(wl, T, x_dev, W_r_dev, bias_dev, n_router, n_experts, 
     router.route(z, wl.k)
     t_router = (time.perf_counter() - t0) * T / len(rows)
 
+    # latent option: x -> latent projection + RMSNorm (and the projection back) per token
+    t_lat = 0.0
+    xe = x                                       # what the experts read
+    if wl.d_latent:
+        W_ld, gamma, W_lu = (t.float().cpu().numpy().astype(np.float64)
+                             for t in synth.draw_latent(wl, device=x_dev.device.type))
+        lrows = rows[:min(n_shared, len(rows))]
+        t0 = time.perf_counter()
+        xn = mx.bf16_round(layer.rms_norm(x[lrows] @ W_ld.T, gamma))
+        mx.bf16_round(xn) @ W_lu.T
+        t_lat = (time.perf_counter() - t0) * T / len(lrows)
+        # the experts' inputs: the latent rows of a token sample (enough for the mean load)
+        xe = np.zeros((T, wl.d_latent))
+        xe[lrows] = xn
+
     load = max(1, int(round(T * wl.k / wl.E)))
     t_exp = 0.0
     for i in range(n_experts):
         e = int(g.integers(wl.E))
         masters = [t.cpu().numpy() for t in synth.draw_expert(wl, e, device=x_dev.device.type)]
-        tok = g.choice(T, size=load, replace=True)
+        tok = g.choice(rows[:min(n_shared, len(rows))] if wl.d_latent else np.arange(T), size=load, replace=True)
         t0 = time.perf_counter()
         Wg, Wu, Wd = layer.decode_expert(layer.quantize_expert(*masters))
-        xq, xs = mx.quantize_mx(x[tok], "e4m3")
+        xq, xs = mx.quantize_mx(xe[tok], "e4m3")
         layer.expert_forward(mx.dequantize_mx(xq, xs, "e4m3"), Wg, Wu, Wd)
         t_exp += time.perf_counter() - t0
     t_exp *= wl.E / max(n_experts, 1)
@@ -103,9 +118,10 @@ def oracle_sample_seconds(wl, T, x_dev, W_r_dev, bias_dev, n_router, n_experts, 
         layer.shared_expert(x[srows], *sw)
         t_sh = (time.perf_counter() - t0) * T / len(srows)
     desc = (f"router on {len(rows)} of {T} tokens, {n_experts} of {wl.E} experts at the mean "
-            f"load of {load} rows (weights quantised+decoded per expert), shared expert on "
+            f"load of {load} rows (weights quantised+decoded per expert), shared expert"
+            f"{' and latent projections' if wl.d_latent else ''} on "
             f"{min(n_shared, len(rows))} tokens; each part scaled linearly to T={T}")
-    return t_router + t_exp + t_sh, desc
+    return t_router + t_exp + t_sh + t_lat, desc
 
 
 # ---------------------------------------------------------------- clocks
@@ -179,8 +195,8 @@ def setup(wl, T, device):
     from block_scaled_moe_sigmoid_b200 import api, synth
     x = synth.draw_x(wl, T, device=device)
     W_r, bias = synth.draw_router(wl, device=device)
-    plan = api.Plan(T, wl.d, wl.E, wl.k, wl.I, wl.I_shared, device=device)
-    ex = api.Experts(wl.d, wl.I, wl.E, device=device)
+    plan = api.Plan(T, wl.d, wl.E, wl.k, wl.I, wl.I_shared, device=device, d_latent=wl.d_latent)
+    ex = api.Experts(wl.d_expert, wl.I, wl.E, device=device)
     for e in range(wl.E):
         g, u, dn = synth.draw_expert(wl, e, device=device)
         ex.pack(e, g, u, dn)
@@ -189,7 +205,11 @@ def setup(wl, T, device):
     if wl.I_shared:
         sh = api.Shared(wl.d, wl.I_shared, device=device)
         sh.pack(*synth.draw_shared(wl, device=device))
+    lat = None
+    if wl.d_latent:
+        lat = api.Latent(*synth.draw_latent(wl, device=device))
     torch.cuda.synchronize()
+    plan.latent = lat
     return x, W_r, bias, plan, ex, sh
 
 
@@ -211,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
 
     def one_step():
         api.moe_route(plan.handle, x, W_r, bias, wl.k, idx=idx, w=w)
-        api.moe_forward(plan.handle, x, idx, w, ex, sh, y)
+        plan.forward(x, idx, w, ex, sh, y, latent=plan.latent)
 
     for _ in range(args.warmup):
         one_step()
@@ -259,7 +279,7 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(max(1, args.warmup)):
             x_dev.copy_(x_host, non_blocking=True)
             api.moe_route(plan.handle, x_dev, W_r, bias, wl.k, idx=idx, w=w)
-            api.moe_forward(plan.handle, x_dev, idx, w, ex, sh, y)
+            plan.forward(x_dev, idx, w, ex, sh, y, latent=plan.latent)
             y_host.copy_(y, non_blocking=True)
         barrier()
         torch.cuda.synchronize()
@@ -268,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(args.steps):
             x_dev.copy_(x_host, non_blocking=True)
             api.moe_route(plan.handle, x_dev, W_r, bias, wl.k, idx=idx, w=w)
-            api.moe_forward(plan.handle, x_dev, idx, w, ex, sh, y)
+            plan.forward(x_dev, idx, w, ex, sh, y, latent=plan.latent)
             y_host.copy_(y, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -296,9 +316,10 @@ def run_ours(args, rank, world, local_rank):
     gu_ms, gu_n = stages["gate_up_glu"]
     t_launch = gu_ms / gu_n / 1e3 if gu_n else None
     A = T * wl.k
-    flops = 2.0 * A * wl.d * (2 * wl.I)
-    gu_bytes = (touched * 2 * wl.I * wl.d * 17 / 32          # E2M1 codes + E8M0 scales
-                + A * wl.d * 33 / 32 + A * wl.I * 33 / 32)     # MXFP8 rows in, GLU rows out
+    de = wl.d_expert                                           # expert input width (d, or d_latent)
+    flops = 2.0 * A * de * (2 * wl.I)
+    gu_bytes = (touched * 2 * wl.I * de * 17 / 32             # E2M1 codes + E8M0 scales
+                + A * de * 33 / 32 + A * wl.I * 33 / 32)       # MXFP8 rows in, GLU rows out
     tc_peak = 2.0 * bf16
     tensor_bound = flops / tc_peak / 1e12 >= gu_bytes / hbm / 1e9
     if tensor_bound:
@@ -321,8 +342,8 @@ def run_ours(args, rank, world, local_rank):
                 "frac_of_nominal_fp4_rate": (flops / t_launch / 1e12 / (4.0 * bf16)) if t_launch else None,
                 "fp4_note": "FP4-rate MMAs (kind::mxf4) need both operands in E2M1; MXFP8 "
                             "activations run at the FP8 rate, so the FP4 figure is context"}
-    w_bytes = (touched * 3 * wl.d * wl.I * 17 / 32 + 3 * wl.d * wl.I_shared * 2
-               + wl.d * wl.E * 4)
+    w_bytes = (touched * 3 * de * wl.I * 17 / 32 + 3 * wl.d * wl.I_shared * 2
+               + wl.d * wl.E * 4 + 2 * wl.d * wl.d_latent * 2)
     stage_ms = {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()}
 
     out = None
@@ -333,7 +354,8 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4xmxfp8 (fp32 acc); bf16 shared/router",
             "data": "synthetic (seeded N(0,1) x, N(0,0.02) weights, random-init)",
-            "config": {"workload": args.workload, "T": T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I,
+            "config": {"workload": args.workload, "T": T, "d": wl.d, "d_latent": wl.d_latent, "E": wl.E,
+                       "k": wl.k, "I": wl.I,
                        "I_shared": wl.I_shared, "seed": wl.seed, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2: every step streams "
                              f"{w_bytes / 1e9:.1f} GB of weights ({touched} touched experts)"},

@@ -36,6 +36,8 @@ SIGNATURES = {
     "moe_pack_shared_bf16": [_I, _I, _P, _P, _P, _P, _P],
     "moe_debug_buffer": [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_S)],
     "moe_debug_timeout_probe": [_P, _P],
+    "moe_plan_set_latent": [_P, _I, ctypes.c_float],
+    "moe_forward_latent": [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P],
     "moe_plan_set_profiling": [_P, _I],
     "moe_plan_set_option": [_P, _I, _I],
     "moe_plan_get_option": [_P, _I, ctypes.POINTER(_I)],
@@ -44,10 +46,10 @@ SIGNATURES = {
 }
 
 STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "gate_up_glu",
-          "down", "shared_gate_up", "shared_down", "combine"]
+          "down", "shared_gate_up", "shared_down", "combine", "latent_in", "latent_out"]
 # kernel launches per recorded stage instance (router_gemm: +1 for the partial-sum kernel
 # when moe_plan_get_option(MOE_OPT_ROUTER_SPLIT) > 1)
-STAGE_KERNELS = {"permute": 3, "quant_scatter": 2}
+STAGE_KERNELS = {"permute": 3, "quant_scatter": 2, "latent_in": 2, "latent_out": 2}
 
 
 class MoeError(RuntimeError):
@@ -62,6 +64,10 @@ class ExpertsMXFP4(ctypes.Structure):
 
 class SharedBF16(ctypes.Structure):
     _fields_ = [("w_gu", _P), ("w_dn", _P)]
+
+
+class LatentBF16(ctypes.Structure):
+    _fields_ = [("w_down", _P), ("gamma", _P), ("w_up", _P)]
 
 
 _lib = None
@@ -185,6 +191,17 @@ def moe_forward(plan, x, idx, w, experts, shared, y=None, stream=None):
     return y
 
 
+def moe_forward_latent(plan, x, idx, w, latent, experts, shared, y=None, stream=None):
+    T, d = x.shape
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device) if y is None else y
+    lat = latent.struct()
+    ex = experts.struct()
+    sh = shared.struct() if shared is not None else None
+    _call("moe_forward_latent", plan, _ptr(x), T, _ptr(idx), _ptr(w), ctypes.byref(lat), ctypes.byref(ex),
+          ctypes.byref(sh) if sh is not None else None, _ptr(y), _stream(stream))
+    return y
+
+
 def moe_expert_bytes(d, I, E):
     a, b, c, e = (ctypes.c_size_t() for _ in range(4))
     _call("moe_expert_bytes", d, I, E, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(e))
@@ -275,14 +292,29 @@ MOE_BIAS_LOGIT, MOE_BIAS_SELECT_ONLY = 0, 1
 MOE_FLAG_STATIC_ROUTER = 1
 
 
+class Latent:
+    """Latent-option weights on the device: W_ld bf16 [d_latent][d], gamma fp32 [d_latent],
+    W_lu bf16 [d][d_latent]."""
+
+    def __init__(self, w_down, gamma, w_up):
+        self.w_down = w_down.to(torch.bfloat16).contiguous()
+        self.gamma = gamma.to(torch.float32).contiguous()
+        self.w_up = w_up.to(torch.bfloat16).contiguous()
+
+    def struct(self):
+        return LatentBF16(self.w_down.data_ptr(), self.gamma.data_ptr(), self.w_up.data_ptr())
+
+
 class Plan:
     """A plan plus its torch-allocated workspace."""
 
     def __init__(self, T_max, d, E, k, I, I_shared=0, device="cuda", act=MOE_ACT_SILU_GLU,
-                 bias_mode=MOE_BIAS_LOGIT, flags=0):
+                 bias_mode=MOE_BIAS_LOGIT, flags=0, d_latent=0, eps=1e-5):
         self.T_max, self.d, self.E, self.k, self.I, self.I_shared = T_max, d, E, k, I, I_shared
-        self.act, self.bias_mode, self.flags = act, bias_mode, flags
+        self.act, self.bias_mode, self.flags, self.d_latent = act, bias_mode, flags, d_latent
         self.handle = moe_plan_create(T_max, d, E, k, I, I_shared, act, bias_mode, flags)
+        if d_latent:
+            _call("moe_plan_set_latent", self.handle, d_latent, ctypes.c_float(eps))
         n = moe_plan_workspace_bytes(self.handle)
         self.workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
         moe_plan_set_workspace(self.handle, self.workspace)
@@ -293,7 +325,9 @@ class Plan:
     def permute(self, idx, stream=None):
         return moe_permute(self.handle, idx, self.E, stream)
 
-    def forward(self, x, idx, w, experts, shared=None, y=None, stream=None):
+    def forward(self, x, idx, w, experts, shared=None, y=None, stream=None, latent=None):
+        if self.d_latent:
+            return moe_forward_latent(self.handle, x, idx, w, latent, experts, shared, y, stream)
         return moe_forward(self.handle, x, idx, w, experts, shared, y, stream)
 
     def check(self, stream=None):

@@ -136,7 +136,9 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
   size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
-      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, total;
+      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_xl, o_xn, o_yl, o_yr, total;
+  int dl = 0;              // latent option: expert width (0 = off)
+  float eps_lat = 1e-5f;
   int tokens_per_chunk() const { return kPermThreads; }
   int nchunks(int T) const { return (T + kPermThreads - 1) / kPermThreads; }
   template <class P>
@@ -170,6 +172,14 @@ static void carve(moe_plan_s* p) {
   p->o_O = take(A * p->d * 2);
   p->o_hsh = take((size_t)p->T_max * (p->Is ? p->Is : 1) * 2);
   p->o_ys = take((size_t)p->T_max * p->d * 4);
+  if (p->dl > 0) {   // latent option: x_l fp32, x_n bf16, y_l bf16 [T][dl], y_r fp32 [T][d]
+    p->o_xl = take((size_t)p->T_max * p->dl * 4);
+    p->o_xn = take((size_t)p->T_max * p->dl * 2);
+    p->o_yl = take((size_t)p->T_max * p->dl * 2);
+    p->o_yr = take((size_t)p->T_max * p->d * 4);
+  } else {
+    p->o_xl = p->o_xn = p->o_yl = p->o_yr = 0;
+  }
   p->total = o;
 }
 
@@ -438,8 +448,31 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   return MOE_OK;
 }
 
-moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx, const float* w,
-                         const moe_experts_mxfp4* ex, const moe_shared_bf16* sh, void* y, void* stream) {
+// A dense bf16 GEMM of the latent option: out fp32 [T][M] = act [T][K] . W [M][K]^T.
+static cudaError_t dense_bf16_f32(const moe_plan_s* p, const void* W, int M, const void* act, int K, int T,
+                                  float* out, int bn, cudaStream_t s) {
+  CUtensorMap tA;
+  BMaps tB;
+  if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, K, M, (uint64_t)K * 2, 64, 256) ||
+      !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act, K, T, (uint64_t)K * 2, 64))
+    return cudaErrorInvalidValue;
+  GemmArgs a = base_args(p);
+  a.dense_rows = T;
+  a.num_groups = 1;
+  a.M_total = M;
+  a.m_tiles = (M + 255) / 256;
+  a.k_tiles = K / 64;
+  a.kb_wrap = a.k_tiles;
+  a.B_rows = T;
+  a.out0 = out;
+  a.ld_out = M;
+  const int tiles = ((T + bn - 1) / bn) * a.m_tiles;
+  return launch_gemm<KIND_BF16, EPI_F32>(bn, a, tA, tB, std::min(tiles, p->num_sms), s);
+}
+
+static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32_t* idx, const float* w,
+                                 const moe_latent_bf16* lat, const moe_experts_mxfp4* ex,
+                                 const moe_shared_bf16* sh, void* y, void* stream) {
   if (!p) return MOE_ERR_INVALID_ARG;
   if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
   if (T < 0) return MOE_ERR_INVALID_ARG;
@@ -453,10 +486,28 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
       !aligned(ex->s_gu, 16) || !aligned(ex->s_dn, 16) ||
       (sh && (!aligned(sh->w_gu, 16) || !aligned(sh->w_dn, 16))))
     return MOE_ERR_ALIGNMENT;
+  if ((lat != nullptr) != (p->dl > 0)) return MOE_ERR_INVALID_ARG;
+  if (lat && (!lat->w_down || !lat->gamma || !lat->w_up)) return MOE_ERR_INVALID_ARG;
+  if (lat && (!aligned(lat->w_down, 16) || !aligned(lat->w_up, 16) || !aligned(lat->gamma, 4)))
+    return MOE_ERR_ALIGNMENT;
   cudaStream_t s = S(stream);
   const int d = p->d, E = p->E, k = p->k, I = p->I, Is = p->Is;
+  const int de = lat ? p->dl : d;   // width the routed experts act on
   const int A = T * k;
   const int bn = p->tile_rows(T);
+
+  // latent option: x_l = x W_ld^T, x_n = bf16(RMSNorm(x_l) * gamma) feeds the experts
+  const void* xin = x;
+  if (lat) {
+    float* xl = p->at<float>(p->o_xl);
+    __nv_bfloat16* xn = p->at<__nv_bfloat16>(p->o_xn);
+    p->prof.begin(MOE_STAGE_LATENT_IN, s);
+    if (dense_bf16_f32(p, lat->w_down, de, x, d, T, xl, bn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    rmsnorm_bf16_kernel<<<T, 256, 0, s>>>(xl, lat->gamma, de, p->eps_lat, xn);
+    p->prof.end(s);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    xin = xn;
+  }
 
   // a4: group assignments by expert
   p->prof.begin(MOE_STAGE_PERMUTE, s);
@@ -466,14 +517,14 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
   uint8_t* xq = p->at<uint8_t>(p->o_xq);
   uint8_t* xs = p->at<uint8_t>(p->o_xs);
   {
-    const long long n = (long long)T * (d / 32);
+    const long long n = (long long)T * (de / 32);
     p->prof.begin(MOE_STAGE_QUANT, s);
     uint8_t* xs_tok = p->at<uint8_t>(p->o_xs_tok);
     quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-        (const uint16_t*)x, T, d, k, p->at<int>(p->o_inv), A, xq, xs_tok);
+        (const uint16_t*)xin, T, de, k, p->at<int>(p->o_inv), A, xq, xs_tok);
     const int max_gt = A / bn + E + 1;   // bound on the group-tiles of this call
-    scale_tiles_kernel<<<max_gt, 256, 0, s>>>(xs_tok, d / 32, p->at<int>(p->o_perm), p->at<int>(p->o_counts),
-                                              p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), E, d / 128, xs);
+    scale_tiles_kernel<<<max_gt, 256, 0, s>>>(xs_tok, de / 32, p->at<int>(p->o_perm), p->at<int>(p->o_counts),
+                                              p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), E, de / 128, xs);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -485,8 +536,8 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     CUtensorMap tA;
     BMaps tB;
     // tile-major weights: 128-element rows of 64 B, one 256-row box per (expert, m-tile, k-tile)
-    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, 128, (uint64_t)E * 2 * I * (d / 128), 64, 128, 256) ||
-        !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, d, A, d, 128))
+    if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_gu, 128, (uint64_t)E * 2 * I * (de / 128), 64, 128, 256) ||
+        !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, de, A, de, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
     a.counts = p->at<int>(p->o_counts);
@@ -495,7 +546,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.num_groups = E;
     a.M_total = 2 * I;
     a.m_tiles = 2 * I / 256;
-    a.k_tiles = d / 128;
+    a.k_tiles = de / 128;
     a.kb_wrap = a.k_tiles;
     a.B_rows = A;
     a.sfa = (const uint8_t*)ex->s_gu;
@@ -516,7 +567,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     CUtensorMap tA;
     BMaps tB;
     if (!make_map(&tA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, ex->w_dn, 128,
-                  (uint64_t)E * ((d + 255) / 256) * 256 * (I / 128), 64, 128, 256) ||
+                  (uint64_t)E * ((de + 255) / 256) * 256 * (I / 128), 64, 128, 256) ||
         !make_bmaps(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, A, I, 128))
       return MOE_ERR_CUDA;
     GemmArgs a = base_args(p);
@@ -524,8 +575,8 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.offsets = p->at<int>(p->o_offsets);
     a.tile_prefix = p->at<int>(p->o_tiles);
     a.num_groups = E;
-    a.M_total = d;
-    a.m_tiles = (d + 255) / 256;
+    a.M_total = de;
+    a.m_tiles = (de + 255) / 256;
     a.k_tiles = I / 128;
     a.kb_wrap = a.k_tiles;
     a.B_rows = A;
@@ -533,7 +584,7 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
     a.a_ptr = (const uint8_t*)ex->w_dn;
     a.sfb = hs;
     a.out0 = O;
-    a.ld_out = d;
+    a.ld_out = de;
     p->prof.begin(MOE_STAGE_DOWN, s);
     if (launch_gemm<KIND_MX, EPI_BF16>(bn, a, tA, tB, p->num_sms, s) != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
@@ -587,14 +638,53 @@ moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx,
       return MOE_ERR_CUDA;
     p->prof.end(s);
   }
-  // a9: weighted combine with the shared output
-  p->prof.begin(MOE_STAGE_COMBINE, s);
-  combine_kernel<<<dim3(T, (d + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
-      O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
-  p->prof.end(s);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (!lat) {
+    // a9: weighted combine with the shared output
+    p->prof.begin(MOE_STAGE_COMBINE, s);
+    combine_kernel<<<dim3(T, (d + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
+        O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
+    p->prof.end(s);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    // latent option: y_l = bf16(sum_j w_j O_j) in the latent, y = bf16(y_l W_lu^T + y_s)
+    __nv_bfloat16* yl = p->at<__nv_bfloat16>(p->o_yl);
+    float* yr = p->at<float>(p->o_yr);
+    p->prof.begin(MOE_STAGE_COMBINE, s);
+    combine_kernel<<<dim3(T, (de + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
+        O, nullptr, w, p->at<int>(p->o_inv), T, de, k, yl);
+    p->prof.end(s);
+    p->prof.begin(MOE_STAGE_LATENT_OUT, s);
+    if (dense_bf16_f32(p, lat->w_up, d, yl, de, T, yr, bn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const long long n = (long long)T * d;
+    add_bf16_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, s>>>(yr, ys, n, (__nv_bfloat16*)y);
+    p->prof.end(s);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
   p->last_T = T;
   p->last_bn = bn;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(moe_plan_t p, const void* x, int T, const int32_t* idx, const float* w,
+                         const moe_experts_mxfp4* ex, const moe_shared_bf16* sh, void* y, void* stream) {
+  if (p && p->dl > 0) return MOE_ERR_INVALID_ARG;   // a latent plan takes moe_forward_latent
+  return forward_impl(p, x, T, idx, w, nullptr, ex, sh, y, stream);
+}
+
+moe_status_t moe_forward_latent(moe_plan_t p, const void* x, int T, const int32_t* idx, const float* w,
+                                const moe_latent_bf16* latent, const moe_experts_mxfp4* ex,
+                                const moe_shared_bf16* sh, void* y, void* stream) {
+  if (!latent) return MOE_ERR_INVALID_ARG;
+  return forward_impl(p, x, T, idx, w, latent, ex, sh, y, stream);
+}
+
+moe_status_t moe_plan_set_latent(moe_plan_t p, int d_latent, float eps) {
+  if (!p || p->ws) return MOE_ERR_INVALID_ARG;
+  if (d_latent <= 0 || d_latent > p->d || eps <= 0.0f) return MOE_ERR_INVALID_ARG;
+  if (d_latent % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  p->dl = d_latent;
+  p->eps_lat = eps;
+  carve(p);
   return MOE_OK;
 }
 

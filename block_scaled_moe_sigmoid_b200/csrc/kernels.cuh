@@ -404,6 +404,45 @@ __global__ void __launch_bounds__(kCombineThreads)
   *(uint4*)(y + (size_t)t * d + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// ---------------------------------------------------------------- latent option
+// x_n[t] = bf16(x_l[t] / sqrt(mean(x_l[t]^2) + eps) * gamma), one CTA (256 threads) per row;
+// the sum of squares in fp32, reduced in a fixed order (per thread, then warp, then CTA).
+__global__ void __launch_bounds__(256)
+    rmsnorm_bf16_kernel(const float* __restrict__ xl, const float* __restrict__ gamma, int cols, float eps,
+                        __nv_bfloat16* __restrict__ xn) {
+  const float* row = xl + (size_t)blockIdx.x * cols;
+  float ss = 0.0f;
+  for (int c = threadIdx.x; c < cols; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  __shared__ float part[8];
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += part[i];
+  const float inv = rsqrtf(tot / (float)cols + eps);
+  for (int c = threadIdx.x; c < cols; c += blockDim.x)
+    xn[(size_t)blockIdx.x * cols + c] = __float2bfloat16_rn(row[c] * inv * __ldg(gamma + c));
+}
+
+// y = bf16(a + b) (b may be NULL), fp32 inputs, 4 elements per thread (n % 4 == 0).
+__global__ void add_bf16_kernel(const float* __restrict__ a, const float* __restrict__ b, long long n,
+                                __nv_bfloat16* __restrict__ y) {
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i >= n) return;
+  float4 v = __ldg((const float4*)(a + i));
+  if (b) {
+    const float4 u = __ldg((const float4*)(b + i));
+    v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 o;
+  o.x = *(const uint32_t*)&lo;
+  o.y = *(const uint32_t*)&hi;
+  *(uint2*)(y + i) = o;
+}
+
 // ---------------------------------------------------------------- failure-path probe
 // One thread waits on an mbarrier of count 1 that nothing arrives at, with the bounded
 // wait of the production kernels; it gives up after the limit and flags the status word.

@@ -20,6 +20,9 @@ Distributions (the workload table of the layer's specification):
   shared W_gate, W_up [I_s, d], W_down [d, I_s] ~ N(0, 0.02) rounded to bf16
   skewed-load bias b_e = 2.0 * ln(1 / (rank_e + 1)^1.2) = -2.4 ln(rank_e + 1),
          rank = a seeded random permutation of 0..E-1
+  latent option (d_latent > 0): experts act on d_latent; projections W_ld [d_latent, d]
+         and W_lu [d, d_latent] ~ N(0, 0.02) rounded to bf16; the RMSNorm gain
+         gamma [d_latent] = 1 + N(0, 0.1) fp32 (the spec gives no distribution)
 The std 0.02 is the config's initializer_range ("Kimi K3" (llm-atlas), raw
 config fields).
 """
@@ -33,6 +36,7 @@ STD = 0.02
 TID_X, TID_WR, TID_RANK = 0, 1, 2
 TID_GATE, TID_UP, TID_DOWN = 3, 4, 5
 TID_SGATE, TID_SUP, TID_SDOWN = 6, 7, 8
+TID_LDOWN, TID_LUP, TID_LGAMMA = 9, 10, 11
 
 
 def stream_seed(seed, tid, sub=0):
@@ -67,6 +71,11 @@ class Workload:
     skew_bias: bool = False
     device: str = "cpu"      # where the generator runs
     sweep: tuple = field(default_factory=tuple)
+    d_latent: int = 0        # > 0: the latent option (experts act on d_latent)
+
+    @property
+    def d_expert(self):
+        return self.d_latent or self.d
 
 
 WORKLOADS = {
@@ -85,6 +94,9 @@ WORKLOADS = {
     # intermediate size 6144 ("Kimi K3.1 Pro vs gpt-oss-120b", component table, shared-expert row)
     "k3_prefill_t8192_shared6144": Workload("k3_prefill_t8192_shared6144", 2, 8192, 7168, 896, 16, 3072, 6144,
                                             device="cuda"),
+    # the latent option at Kimi-K3 shape: experts on a 3584-dim latent (half of d)
+    "k3_latent_prefill_t8192": Workload("k3_latent_prefill_t8192", 2, 8192, 7168, 896, 16, 3072, 3072,
+                                        device="cuda", d_latent=3584),
     # token-count sweep (T is given per run)
     "k3_sweep": Workload("k3_sweep", 4, 1, 7168, 896, 16, 3072, 3072, device="cuda",
                          sweep=(1, 16, 256, 2048, 16384)),
@@ -111,11 +123,24 @@ def draw_router(wl, device=None):
 
 
 def draw_expert(wl, e, device=None):
-    """fp32 masters of expert e: (W_gate [I, d], W_up [I, d], W_down [d, I])."""
+    """fp32 masters of expert e: (W_gate [I, de], W_up [I, de], W_down [de, I]) with
+    de = d, or d_latent for the latent option."""
     dev = wl.device if device is None else device
-    return (normal((wl.I, wl.d), wl.seed, TID_GATE, e, STD, dev),
-            normal((wl.I, wl.d), wl.seed, TID_UP, e, STD, dev),
-            normal((wl.d, wl.I), wl.seed, TID_DOWN, e, STD, dev))
+    de = wl.d_expert
+    return (normal((wl.I, de), wl.seed, TID_GATE, e, STD, dev),
+            normal((wl.I, de), wl.seed, TID_UP, e, STD, dev),
+            normal((de, wl.I), wl.seed, TID_DOWN, e, STD, dev))
+
+
+def draw_latent(wl, device=None):
+    """Latent option: (W_ld bf16 [d_latent, d], gamma fp32 [d_latent], W_lu bf16 [d, d_latent])."""
+    if not wl.d_latent:
+        return None
+    dev = wl.device if device is None else device
+    dl = wl.d_latent
+    gamma = normal((dl,), wl.seed, TID_LGAMMA, 0, 0.1, dev).add_(1.0)
+    return (normal((dl, wl.d), wl.seed, TID_LDOWN, 0, STD, dev).to(torch.bfloat16), gamma,
+            normal((wl.d, dl), wl.seed, TID_LUP, 0, STD, dev).to(torch.bfloat16))
 
 
 def draw_shared(wl, device=None):
@@ -130,6 +155,6 @@ def draw_shared(wl, device=None):
 
 
 def custom(name="custom", seed=0, T=8, d=256, E=8, k=2, I=128, I_shared=0,
-           skew_bias=False, device="cpu"):
+           skew_bias=False, device="cpu", d_latent=0):
     """A workload of arbitrary (small) shape for tests."""
-    return Workload(name, seed, T, d, E, k, I, I_shared, skew_bias, device)
+    return Workload(name, seed, T, d, E, k, I, I_shared, skew_bias, device, d_latent=d_latent)

@@ -181,6 +181,32 @@ moe_status_t moe_forward(moe_plan_t plan, const void* x_bf16, int T, const int32
                          const float* w, const moe_experts_mxfp4* experts,
                          const moe_shared_bf16* shared, void* y_bf16, void* stream);
 
+/* ---- latent option ---------------------------------------------------------------------
+ * Reading of the pages' "Stable LatentMoE": the routed experts run on a d_latent-wide
+ * latent with an RMSNorm before them ("Kimi K3.1 Pro vs gpt-oss-120b" and "Gemma 4 31B vs
+ * Kimi K3", component tables, routed-experts row; "Kimi K3" (llm-atlas), raw config:
+ * routed_expert_hidden_size 3584, latent_moe_use_norm, rms_norm_eps 1e-5).  The pages do
+ * not publish where the projections sit, so this is the plainest reading:
+ *   x_l = x W_ld^T (bf16 x bf16, fp32 accumulation)
+ *   x_n = bf16(x_l / sqrt(mean(x_l^2) + eps) * gamma)
+ *   y_l = bf16(sum_j w[t][j] * expert_{idx[t][j]}(x_n))   (experts packed with d = d_latent)
+ *   y   = bf16(y_l W_lu^T + shared(x))                    (fp32 sum; shared reads x itself)
+ * moe_plan_set_latent: d_latent % 128 == 0 and 0 < d_latent <= d; eps > 0.  Call it before
+ * moe_plan_workspace_bytes / moe_plan_set_workspace (the workspace grows by the latent
+ * buffers); MOE_ERR_INVALID_ARG once a workspace is attached. */
+typedef struct {
+  const void* w_down;   /* bf16 [d_latent][d]: x -> latent (device) */
+  const float* gamma;   /* fp32 [d_latent]: RMSNorm gain (device) */
+  const void* w_up;     /* bf16 [d][d_latent]: latent -> d (device) */
+} moe_latent_bf16;
+moe_status_t moe_plan_set_latent(moe_plan_t plan, int d_latent, float eps);
+/* The layer with the latent option; arguments as moe_forward plus `latent`.  The plan
+ * must have had moe_plan_set_latent; experts are packed with d = d_latent. */
+moe_status_t moe_forward_latent(moe_plan_t plan, const void* x_bf16, int T, const int32_t* idx,
+                                const float* w, const moe_latent_bf16* latent,
+                                const moe_experts_mxfp4* experts, const moe_shared_bf16* shared,
+                                void* y_bf16, void* stream);
+
 /* ---- setup helpers (not on the timed path) --------------------------------------------
  * Byte sizes of the four packed expert arrays for E experts (host outputs). */
 moe_status_t moe_expert_bytes(int d, int I, int E, size_t* w_gu, size_t* s_gu, size_t* w_dn,
@@ -233,7 +259,9 @@ enum {
   MOE_STAGE_SHARED_GATE_UP = 7,  /* shared expert gate/up + GLU */
   MOE_STAGE_SHARED_DOWN = 8,     /* shared expert down */
   MOE_STAGE_COMBINE = 9,         /* weighted combine */
-  MOE_NUM_STAGES = 10
+  MOE_STAGE_LATENT_IN = 10,      /* latent option: x -> latent GEMM + RMSNorm (2 kernels) */
+  MOE_STAGE_LATENT_OUT = 11,     /* latent option: latent -> d GEMM + final add (2 kernels) */
+  MOE_NUM_STAGES = 12
 };
 moe_status_t moe_plan_set_profiling(moe_plan_t plan, int enable);
 moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n);

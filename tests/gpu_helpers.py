@@ -89,8 +89,11 @@ class Case:
         self.W_r, self.bias = W_r.to(dev).contiguous(), b.to(dev).contiguous()
         self.plan = api.Plan(max(self.T, 1), wl.d, wl.E, wl.k, wl.I, wl.I_shared,
                              act={"silu": api.MOE_ACT_SILU_GLU, "clamped_swiglu": api.MOE_ACT_CLAMPED_SWIGLU}[act],
-                             bias_mode=api.MOE_BIAS_SELECT_ONLY if select_only else api.MOE_BIAS_LOGIT)
-        self.experts = api.Experts(wl.d, wl.I, wl.E)
+                             bias_mode=api.MOE_BIAS_SELECT_ONLY if select_only else api.MOE_BIAS_LOGIT,
+                             d_latent=wl.d_latent)
+        self.latent_w = synth.draw_latent(wl, device=gd)
+        self.latent = api.Latent(*(t.to(dev) for t in self.latent_w)) if self.latent_w else None
+        self.experts = api.Experts(wl.d_expert, wl.I, wl.E)
         for e in range(wl.E):
             g, u, dn = (t.to(dev) for t in synth.draw_expert(wl, e, device=gd))
             self.experts.pack(e, g, u, dn)
@@ -115,6 +118,11 @@ class Case:
             ms = [t.cpu().numpy() for t in synth.draw_expert(self.wl, e, device=self.gen_device)]
             self._oracle_w[e] = layer.decode_expert(layer.quantize_expert(*ms))
         return self._oracle_w[e]
+
+    def oracle_latent(self):
+        if self.latent_w is None:
+            return None
+        return tuple(t.float().cpu().numpy().astype(np.float64) for t in self.latent_w)
 
     def oracle_shared(self):
         if self.shared_w is None:

@@ -308,6 +308,51 @@ def test_layer_max_top_k_32():
     _check_layer(case, stage_checks=True)
 
 
+def _check_latent_layer(case):
+    idx, w, idx_o, w_o, gap = _check_route(case)
+    y = case.plan.forward(case.x, idx, w, case.experts, case.shared, latent=case.latent)
+    assert case.plan.check()[0] == 0
+    y = y.float().cpu().numpy().astype(np.float64)
+    y_ref = layer.latent_moe_layer(case.x_np(), idx_o, w_o, case.oracle_expert, case.oracle_latent(),
+                                   case.oracle_shared(), act=case.act)
+    st = layer_stats(y, y_ref, gap)
+    assert st["max_rel"] <= MAX_REL and st["mean_rel"] <= MEAN_REL, st
+    return st
+
+
+def test_layer_latent_option():
+    """The latent option (experts on a d/2 latent, RMSNorm before them, projections back),
+    with a shared expert on the un-projected input and a ragged token count."""
+    wl = synth.custom(seed=20, T=150, d=256, E=12, k=3, I=128, I_shared=128, d_latent=128)
+    case = Case(wl)
+    print("latent", _check_latent_layer(case))
+
+
+def test_layer_latent_option_wide_and_small_tiles():
+    """d_latent spanning two 256-row output tiles of the expert down GEMM (d_latent = 384 of
+    d = 512), no shared expert, both GEMM tile configurations."""
+    wl = synth.custom(seed=21, T=64, d=512, E=8, k=2, I=128, d_latent=384)
+    case = Case(wl)
+    for bn in (32, 160):
+        api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, bn)
+        _check_latent_layer(case)
+
+
+def test_latent_plan_rejects_the_plain_call_and_bad_shapes():
+    wl = synth.custom(seed=22, T=8, d=256, E=4, k=2, I=128, d_latent=128)
+    case = Case(wl)
+    idx, w = case.plan.route(case.x, case.W_r, case.bias)
+    with pytest.raises(api.MoeError):
+        api.moe_forward(case.plan.handle, case.x, idx, w, case.experts, None)
+    h = api.moe_plan_create(8, 256, 4, 2, 128)
+    L = api.lib()
+    import ctypes
+    assert L.moe_plan_set_latent(h, 100, ctypes.c_float(1e-5)) == 2     # not a multiple of 128
+    assert L.moe_plan_set_latent(h, 384, ctypes.c_float(1e-5)) == 1     # wider than d
+    assert L.moe_plan_set_latent(h, 128, ctypes.c_float(0.0)) == 1      # eps must be > 0
+    api.moe_plan_destroy(h)
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
