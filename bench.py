@@ -269,6 +269,10 @@ def run_ours(args, rank, world, local_rank):
     launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
     if api.moe_plan_get_option(plan.handle, api.MOE_OPT_ROUTER_SPLIT) > 1:
         launches += stages["router_gemm"][1]   # the K-split partial sum
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1:
+        launches += stages["shared_gate_up"][1]
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT_DOWN) > 1:
+        launches += stages["shared_down"][1]
 
     # ---- end to end through the public API with host buffers
     # Every step copies its input x from pinned host memory and its output y back, inside

@@ -228,6 +228,7 @@ def moe_debug_buffer(plan, which):
 
 
 MOE_OPT_PREFETCH_DIST, MOE_OPT_PREFETCH_B, MOE_OPT_TILE_N, MOE_OPT_ROUTER_SPLIT = 0, 1, 2, 3
+MOE_OPT_SHARED_SPLIT, MOE_OPT_SHARED_SPLIT_DOWN = 4, 5
 
 
 def moe_plan_set_option(plan, option, value):

@@ -28,6 +28,7 @@ constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
 constexpr int kRouterStages = 3;
 constexpr int kRouterMaxCtas = 256;   // bound on split router tiles (sizes the partials)
+constexpr int kSplitMaxCtas = 256;    // bound on split-K dense GEMM tiles (sizes their partials)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -126,6 +127,8 @@ struct moe_plan_s {
   int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
   int last_bn = 0;            // token rows per tile in the last moe_forward
   int last_ksplit = 0;        // router K splits in the last moe_route
+  int last_shared_split = 0;     // shared-expert gate/up K splits in the last moe_forward
+  int last_shared_split_dn = 0;  // shared-expert down K splits in the last moe_forward
   size_t zpart_floats = 0;    // capacity of the router partials
   // token rows per GEMM tile for a call with T tokens
   int tile_rows(int T) const {
@@ -136,7 +139,7 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
   size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
-      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_xl, o_xn, o_yl, o_yr, total;
+      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_spart, o_xl, o_xn, o_yl, o_yr, total;
   int dl = 0;              // latent option: expert width (0 = off)
   float eps_lat = 1e-5f;
   int tokens_per_chunk() const { return kPermThreads; }
@@ -172,6 +175,9 @@ static void carve(moe_plan_s* p) {
   p->o_O = take(A * p->d * 2);
   p->o_hsh = take((size_t)p->T_max * (p->Is ? p->Is : 1) * 2);
   p->o_ys = take((size_t)p->T_max * p->d * 4);
+  // split-K partials of the dense shared-expert GEMMs: ksplit * tiles <= kSplitMaxCtas, so
+  // ksplit * T * M <= kSplitMaxCtas * kBN * 256 floats
+  p->o_spart = take((size_t)kSplitMaxCtas * kBN * 256 * 4);
   if (p->dl > 0) {   // latent option: x_l fp32, x_n bf16, y_l bf16 [T][dl], y_r fp32 [T][d]
     p->o_xl = take((size_t)p->T_max * p->dl * 4);
     p->o_xn = take((size_t)p->T_max * p->dl * 2);
@@ -216,11 +222,26 @@ static cudaError_t launch_gemm(int bn, const GemmArgs& a, const CUtensorMap& tA,
   return launch_gemm_cfg<KIND, EPI, kBN, kStages>(a, tA, tB, grid, s);
 }
 
+// K splits for a dense GEMM with `tiles` output tiles and k_tiles K tiles: when the tiles
+// would fill less than half the SMs (few tokens), split K so that up to one CTA runs per SM,
+// keeping at least 4 K tiles per split and the fp32 partials (ksplit * elems) within the
+// workspace.  1 = no split.  No split is empty: (ks - 1) * ceil(k_tiles / ks) < k_tiles.
+static int dense_ksplit(const moe_plan_s* p, int tiles, int k_tiles, size_t elems) {
+  const int cap = std::min(p->num_sms, kSplitMaxCtas);
+  if (tiles <= 0 || 2 * tiles > cap) return 1;
+  int ks = std::min(cap / tiles, k_tiles / 4);
+  while (ks > 1 && (size_t)ks * elems > (size_t)kSplitMaxCtas * kBN * 256) --ks;
+  if (ks <= 1) return 1;
+  const int per = (k_tiles + ks - 1) / ks;
+  return (k_tiles + per - 1) / per;   // no empty split
+}
+
 static GemmArgs base_args(const moe_plan_s* p) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
   a.status = p->at<unsigned int>(p->o_status);
   a.dense_rows = -1;
+  a.ksplit = 1;
   a.pf_dist = p->pf_dist;
   a.pf_b = p->pf_b;
   return a;
@@ -610,12 +631,32 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     a.out0 = hsh;
     a.ld_out = Is;
     int tiles = ((T + bn - 1) / bn) * a.m_tiles;
+    float* spart = p->at<float>(p->o_spart);
     p->prof.begin(MOE_STAGE_SHARED_GATE_UP, s);
-    const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
-        ? launch_gemm<KIND_BF16, EPI_GLU_BF16_CLAMPED>(bn, a, tA, tB, std::min(tiles, p->num_sms), s)
-        : launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s);
-    if (e != cudaSuccess)
-      return MOE_ERR_CUDA;
+    const int ks_gu = dense_ksplit(p, tiles, a.k_tiles, (size_t)T * 2 * Is);
+    if (ks_gu > 1) {
+      // few token tiles: split K over the SMs, fp32 partials, then sum + GLU + bf16
+      a.ksplit = ks_gu;
+      a.k_per = (a.k_tiles + ks_gu - 1) / ks_gu;
+      a.split_stride = (long long)T * 2 * Is;
+      a.out0 = spart;
+      a.ld_out = 2 * Is;
+      if (launch_gemm<KIND_BF16, EPI_F32>(bn, a, tA, tB, std::min(tiles * ks_gu, p->num_sms), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      const long long n = (long long)T * Is;
+      if (p->act == MOE_ACT_CLAMPED_SWIGLU)
+        split_glu_reduce_kernel<1><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_gu, T, Is, a.split_stride, hsh);
+      else
+        split_glu_reduce_kernel<0><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_gu, T, Is, a.split_stride, hsh);
+      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+      const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
+          ? launch_gemm<KIND_BF16, EPI_GLU_BF16_CLAMPED>(bn, a, tA, tB, std::min(tiles, p->num_sms), s)
+          : launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s);
+      if (e != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    p->last_shared_split = ks_gu;
     p->prof.end(s);
     CUtensorMap tA2;
     BMaps tB2;
@@ -634,9 +675,25 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     b.ld_out = d;
     tiles = ((T + bn - 1) / bn) * b.m_tiles;
     p->prof.begin(MOE_STAGE_SHARED_DOWN, s);
-    if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    const int ks_dn = dense_ksplit(p, tiles, b.k_tiles, (size_t)T * d);
+    if (ks_dn > 1) {
+      b.ksplit = ks_dn;
+      b.k_per = (b.k_tiles + ks_dn - 1) / ks_dn;
+      b.split_stride = (long long)T * d;
+      b.out0 = spart;
+      if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles * ks_dn, p->num_sms), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      const long long n = (long long)T * d;
+      split_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_dn, n, b.split_stride, ys);
+      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+      if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    p->last_shared_split_dn = ks_dn;
     p->prof.end(s);
+  } else {
+    p->last_shared_split = p->last_shared_split_dn = 0;
   }
   if (!lat) {
     // a9: weighted combine with the shared output
@@ -764,6 +821,8 @@ moe_status_t moe_plan_get_option(moe_plan_t p, int option, int* value) {
     case MOE_OPT_PREFETCH_B: *value = p->pf_b; return MOE_OK;
     case MOE_OPT_TILE_N: *value = p->last_bn; return MOE_OK;
     case MOE_OPT_ROUTER_SPLIT: *value = p->last_ksplit; return MOE_OK;
+    case MOE_OPT_SHARED_SPLIT: *value = p->last_shared_split; return MOE_OK;
+    case MOE_OPT_SHARED_SPLIT_DOWN: *value = p->last_shared_split_dn; return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
 }

@@ -69,6 +69,11 @@ struct GemmArgs {
   int pf_dist;          // L2 prefetch distance in k-tiles (0 = off), KIND_MX weights
   int pf_b;             // reserved
   const uint8_t* a_ptr; // KIND_MX: packed weights (base of the tile-major code array)
+  // Split K (dense mode with EPI_F32 only): tiles also walk ksplit ranges of k_per K tiles,
+  // and split s writes its fp32 partial at out0 + s * split_stride elements.
+  int ksplit;
+  int k_per;
+  long long split_stride;
 };
 
 template <int KIND, int BN_MAX, int STAGES>
@@ -97,14 +102,25 @@ struct GemmCfg {
 
 struct TileInfo {
   int grp, gt, mt, row0, n_valid, n_mma;  // gt: group-tile index
+  int split, kb, ke;                       // K split and its K-tile range [kb, ke)
 };
 
 __device__ __forceinline__ int gemm_num_tiles(const GemmArgs& a, int bn_max) {
-  if (a.dense_rows >= 0) return ((a.dense_rows + bn_max - 1) / bn_max) * a.m_tiles;
+  if (a.dense_rows >= 0) return ((a.dense_rows + bn_max - 1) / bn_max) * a.m_tiles * a.ksplit;
   return __ldg(a.tile_prefix + a.num_groups) * a.m_tiles;
 }
 
 __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, int t, TileInfo& ti) {
+  ti.split = 0;
+  ti.kb = 0;
+  ti.ke = a.k_tiles;
+  if (a.dense_rows >= 0 && a.ksplit > 1) {   // the split is the slowest index of t
+    const int per_split = ((a.dense_rows + bn_max - 1) / bn_max) * a.m_tiles;
+    ti.split = t / per_split;
+    t -= ti.split * per_split;
+    ti.kb = ti.split * a.k_per;
+    ti.ke = min(a.k_tiles, ti.kb + a.k_per);
+  }
   const int gt = t / a.m_tiles;
   ti.mt = t - gt * a.m_tiles;
   int grp, nt, ntiles, Me, base;
@@ -138,6 +154,37 @@ __device__ __forceinline__ void gemm_decode_tile(const GemmArgs& a, int bn_max, 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 // a = glu(g, u): ACT 0 SiLU-GLU; ACT 1 clamped SwiGLU, (clamp(u, -7, 7) + 1) * g_c *
 // sigmoid(1.702 g_c) with g_c = min(g, 7)
+template <int ACT>
+__device__ __forceinline__ float glu_f(float g, float u);
+
+// Split-K partials of a gate/up product, rows interleaved in 128-channel blocks (gate
+// block, up block, ...): h[t][c] = bf16(glu(sum_s g, sum_s u)), sums in split order.
+template <int ACT>
+__global__ void split_glu_reduce_kernel(const float* __restrict__ part, int nsplit, int T, int I,
+                                        long long split_stride, __nv_bfloat16* __restrict__ h) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)T * I) return;
+  const int t = (int)(i / I), c = (int)(i - (long long)t * I);
+  const size_t gcol = (size_t)256 * (c >> 7) + (c & 127);
+  const float* row = part + (size_t)t * 2 * I;
+  float g = 0.0f, u = 0.0f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    g += __ldg(row + sp * split_stride + gcol);
+    u += __ldg(row + sp * split_stride + gcol + 128);
+  }
+  h[i] = __float2bfloat16_rn(glu_f<ACT>(g, u));
+}
+
+// out[i] = sum over s, in order, of part[s * split_stride + i].
+__global__ void split_sum_kernel(const float* __restrict__ part, int nsplit, long long n, long long split_stride,
+                                 float* __restrict__ out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float v = 0.0f;
+  for (int sp = 0; sp < nsplit; ++sp) v += __ldg(part + sp * split_stride + i);
+  out[i] = v;
+}
+
 template <int ACT>
 __device__ __forceinline__ float glu_f(float g, float u) {
   if constexpr (ACT == 0) {
@@ -247,7 +294,7 @@ __global__ void __launch_bounds__(384, 1)
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
       const int a_row = ti.grp * args.M_total + ti.mt * C::BM;
-      for (int kt = 0; kt < args.k_tiles; ++kt) {
+      for (int kt = ti.kb; kt < ti.ke; ++kt) {
         if (lane == 0) {
           ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
           if (ok) {
@@ -289,7 +336,7 @@ __global__ void __launch_bounds__(384, 1)
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
       const int nB = (ti.n_mma + 31) >> 5;
-      for (int kt = 0; kt < args.k_tiles; ++kt) {
+      for (int kt = ti.kb; kt < ti.ke; ++kt) {
         if (lane == 0) ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
@@ -332,7 +379,7 @@ __global__ void __launch_bounds__(384, 1)
         gemm_decode_tile(args, BN_MAX, t, ti);
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
         const int atoms = (ti.n_mma + 127) >> 7;
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = ti.kb; kt < ti.ke; ++kt) {
           ok = mbar_wait(smem_u32(sf_full + stage), phase, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
@@ -398,15 +445,15 @@ __global__ void __launch_bounds__(384, 1)
         // MMAs issued in one run.  Each mbarrier wait costs the issuing thread about as much
         // as one or two MMAs even when the stage has long landed, so pairing halves that
         // overhead per MMA.  Each stage is still released as soon as its own MMAs commit.
-        for (int kt = 0; kt < args.k_tiles; kt += 2) {
-          const bool two = kt + 1 < args.k_tiles;
+        for (int kt = ti.kb; kt < ti.ke; kt += 2) {
+          const bool two = kt + 1 < ti.ke;
           const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (ok && two) ok = mbar_wait(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_stage(stage, kt > 0 ? 1u : 0u);
+          issue_stage(stage, kt > ti.kb ? 1u : 0u);
           tc_commit(smem_u32(empty_bar + stage));
           if (two) {
             issue_stage(stage2, 1u);
@@ -540,7 +587,8 @@ __global__ void __launch_bounds__(384, 1)
               const int n = c * 16 + j;
               if (n >= ti.n_valid) break;
               if (!ch_ok) continue;
-              ((float*)args.out0)[(size_t)(ti.row0 + n) * args.ld_out + ch] = __uint_as_float(v[j]);
+              ((float*)args.out0)[(size_t)ti.split * args.split_stride + (size_t)(ti.row0 + n) * args.ld_out + ch] =
+                  __uint_as_float(v[j]);
             }
           }
         }

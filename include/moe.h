@@ -235,10 +235,16 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  *   the router GEMM (1 = none).  With few tokens the router splits d over up to one
  *   CTA per SM and adds the fp32 partials in split order (plus the bias) in one more
  *   kernel, so that call launches 4 kernels instead of 3.
+ * MOE_OPT_SHARED_SPLIT / MOE_OPT_SHARED_SPLIT_DOWN (read only): K splits of the shared
+ *   expert's gate/up and down GEMMs in the last moe_forward (1 = none; 0 without a shared
+ *   expert).  With few tokens these dense GEMMs split K over the SMs.  Each split GEMM writes
+ *   fp32 partials, and one more kernel adds them in split order (the gate/up one also applies
+ *   the GLU), so each split adds one launch.
  * moe_plan_get_option reads an option back (host int); for MOE_OPT_TILE_N it returns the
  * tile rows that the last moe_forward on this plan used (0 before the first call), which
  * fixes the tile-major layout of the token-side scale blocks (debug buffers 1 and 3). */
-enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1, MOE_OPT_TILE_N = 2, MOE_OPT_ROUTER_SPLIT = 3 };
+enum { MOE_OPT_PREFETCH_DIST = 0, MOE_OPT_PREFETCH_B = 1, MOE_OPT_TILE_N = 2, MOE_OPT_ROUTER_SPLIT = 3,
+       MOE_OPT_SHARED_SPLIT = 4, MOE_OPT_SHARED_SPLIT_DOWN = 5 };
 moe_status_t moe_plan_set_option(moe_plan_t plan, int option, int value);
 moe_status_t moe_plan_get_option(moe_plan_t plan, int option, int* value);
 

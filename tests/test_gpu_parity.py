@@ -353,6 +353,22 @@ def test_latent_plan_rejects_the_plain_call_and_bad_shapes():
     api.moe_plan_destroy(h)
 
 
+def test_layer_shared_expert_split_k():
+    """Few tokens and a wide d: the shared expert's dense GEMMs split K over the SMs (fp32
+    partials, then sum + GLU, and sum); the layer still matches the oracle and repeats
+    bit for bit."""
+    wl = synth.custom(seed=23, T=40, d=1024, E=8, k=2, I=128, I_shared=1024)
+    case = Case(wl)
+    st = _check_layer(case)
+    assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1
+    assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_SHARED_SPLIT_DOWN) > 1
+    idx, w = case.plan.route(case.x, case.W_r, case.bias)
+    y1 = case.plan.forward(case.x, idx, w, case.experts, case.shared).clone()
+    y2 = case.plan.forward(case.x, idx, w, case.experts, case.shared)
+    assert torch.equal(y1, y2)
+    print("shared split", st)
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
