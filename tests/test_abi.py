@@ -46,6 +46,23 @@ def test_host_side_argument_checks_without_gpu():
     for act, mode in ((1, 0), (0, 1), (1, 1)):
         assert L.moe_plan_create(16, 128, 8, 2, 128, 0, act, mode, 0, ctypes.byref(h)) == 0
         assert L.moe_plan_destroy(h) == 0
+    # latent option: shape checks on a host-only plan (no workspace attached yet)
+    assert L.moe_plan_create(16, 256, 8, 2, 128, 0, 0, 0, 0, ctypes.byref(h)) == 0
+    assert L.moe_plan_set_latent(h, 100, ctypes.c_float(1e-5)) == 2     # not a multiple of 128
+    assert L.moe_plan_set_latent(h, 384, ctypes.c_float(1e-5)) == 1     # wider than d
+    assert L.moe_plan_set_latent(h, 128, ctypes.c_float(0.0)) == 1      # eps must be > 0
+    n0 = ctypes.c_size_t()
+    assert L.moe_plan_workspace_bytes(h, ctypes.byref(n0)) == 0
+    assert L.moe_plan_set_latent(h, 128, ctypes.c_float(1e-5)) == 0
+    n1 = ctypes.c_size_t()
+    assert L.moe_plan_workspace_bytes(h, ctypes.byref(n1)) == 0
+    assert n1.value > n0.value                                          # latent buffers added
+    v = ctypes.c_int()
+    for opt in (0, 1, 2, 3, 4, 5):
+        assert L.moe_plan_get_option(h, opt, ctypes.byref(v)) == 0
+    assert L.moe_plan_get_option(h, 99, ctypes.byref(v)) == 1
+    assert L.moe_plan_set_option(h, 3, 1) == 1                          # read-only option
+    assert L.moe_plan_destroy(h) == 0
     assert L.moe_quant_mxfp8(None, 4, 33, None, None, None) == 2
     assert L.moe_status_string(3) == b"misaligned pointer"
     sizes = api.moe_expert_bytes(7168, 3072, 896)
