@@ -340,6 +340,13 @@ def run_ours(args, rank, world, local_rank):
         bf16, peak_src = 1400.0, "fallback"
     hbm, hbm_src = (peaks["hbm_gbs"], "measured") if peaks.get("hbm_gbs") else (6650.0, "fallback")
     touched = int(torch.unique(idx).numel())
+    # per-expert load of the timed routing (assignments per expert), summarised
+    load = torch.bincount(idx.reshape(-1).long(), minlength=wl.E).cpu()
+    ls = torch.sort(load, descending=True).values
+    expert_load = {"mean": float(load.float().mean()), "max": int(ls[0]), "min": int(ls[-1]),
+                   "p50": int(ls[wl.E // 2]), "p90": int(ls[wl.E // 10]), "zero_experts": int((load == 0).sum()),
+                   "top8": [int(v) for v in ls[:8]],
+                   "share_of_top_1pct": float(ls[:max(1, wl.E // 100)].sum()) / max(1, int(load.sum()))}
     gu_ms, gu_n = stages["gate_up_glu"]
     t_launch = gu_ms / gu_n / 1e3 if gu_n else None
     A = T * wl.k
@@ -388,6 +395,7 @@ def run_ours(args, rank, world, local_rank):
                              f"{w_bytes / 1e9:.1f} GB of weights ({touched} touched experts)"},
             "roofline": roofline,
             "gemm_tile_rows": api.moe_plan_get_option(plan.handle, api.MOE_OPT_TILE_N),
+            "expert_load": expert_load,
             "hbm_view": {"weight_bytes_per_step": w_bytes, "touched_experts": touched,
                          "achieved_gbs": w_bytes / (ms / args.steps / 1e3) / 1e9,
                          "peak_gbs": hbm, "frac": w_bytes / (ms / args.steps / 1e3) / 1e9 / hbm,
