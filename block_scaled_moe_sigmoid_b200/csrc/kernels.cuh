@@ -95,8 +95,33 @@ __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int 
   for (int i = 0; i < 4; ++i) in[i] = __ldg(src + i);
   uint32_t out[8];
   xs_tok[gid] = (uint8_t)quant_block_e4m3(in, out);
-  const uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
-  const uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
+  uint4 o0 = make_uint4(out[0], out[1], out[2], out[3]);
+  uint4 o1 = make_uint4(out[4], out[5], out[6], out[7]);
+  // When a warp's 32 blocks are one token's 1 KB run (cols % 1024 == 0, so that no warp
+  // straddles two tokens), regroup the codes through shuffles so that each warp-wide store
+  // writes 512 contiguous bytes: lane l stores bytes [16 l, 16 l + 16) and [512 + 16 l, ...)
+  // of the run, i.e. half (l % 2) of blocks l / 2 and 16 + l / 2.  Otherwise lane l stores
+  // its own block's 32 bytes.
+  int boff0 = b * 32, boff1 = b * 32 + 16;
+  if ((nb & 31) == 0) {
+    const int lane = threadIdx.x & 31;
+    const int s0 = lane >> 1, s1 = 16 + (lane >> 1);
+    const bool hi = lane & 1;
+    uint32_t a[4], c[4];
+    const uint32_t w0[4] = {o0.x, o0.y, o0.z, o0.w}, w1[4] = {o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x0 = __shfl_sync(0xffffffffu, w0[i], s0), x1 = __shfl_sync(0xffffffffu, w1[i], s0);
+      const uint32_t y0 = __shfl_sync(0xffffffffu, w0[i], s1), y1 = __shfl_sync(0xffffffffu, w1[i], s1);
+      a[i] = hi ? x1 : x0;
+      c[i] = hi ? y1 : y0;
+    }
+    o0 = make_uint4(a[0], a[1], a[2], a[3]);
+    o1 = make_uint4(c[0], c[1], c[2], c[3]);
+    const int b0 = b & ~31;   // first block of this warp's run
+    boff0 = b0 * 32 + 16 * lane;
+    boff1 = b0 * 32 + 512 + 16 * lane;
+  }
   // four destinations at a time, so that their index loads overlap
   for (int j0 = 0; j0 < k; j0 += 4) {
     int pj[4];
@@ -106,9 +131,9 @@ __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int 
     for (int q = 0; q < 4; ++q) {
       const int p = pj[q];
       if (p < 0 || p >= A_rows) continue;
-      uint4* dst = (uint4*)(xq + (size_t)p * cols + b * 32);
-      dst[0] = o0;
-      dst[1] = o1;
+      uint8_t* row = xq + (size_t)p * cols;
+      *(uint4*)(row + boff0) = o0;
+      *(uint4*)(row + boff1) = o1;
     }
   }
 }
