@@ -369,6 +369,15 @@ def test_layer_shared_expert_split_k():
     print("shared split", st)
 
 
+def test_layer_clamped_swiglu_with_shared_split_k():
+    """The clamped SwiGLU through the split-K shared expert (partials summed, then the
+    clamped GLU in the reduction kernel)."""
+    wl = synth.custom(seed=24, T=40, d=1024, E=8, k=2, I=128, I_shared=1024)
+    case = Case(wl, act="clamped_swiglu", x_scale=8.0)
+    _check_layer(case)
+    assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1
+
+
 def test_layer_dense_mixture_k_equals_e():
     wl = synth.custom(seed=10, T=50, d=256, E=4, k=4, I=128)
     case = Case(wl)
