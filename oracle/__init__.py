@@ -16,7 +16,11 @@ Modules:
   layer    routed expert GLU MLP, MXFP8 requantisation, shared expert, combine
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``.
-The parts that the pages leave unpinned are SiTU, Quantile Balancing and the
-latent projection.  They are not implemented, so nothing here is marked
-"parity unpinned".
+SiTU has no published formula and is not implemented.  The latent option
+(``layer.latent_moe_layer``, reading R22) is implemented; where its projections
+sit is a reading, not something the pages fix, and it is pinned against a
+torch restatement of that same reading.  The Quantile Balancing update rule is
+unpublished: ``router.routing_margins`` and ``router.margin_quantiles`` compute
+the margins and quantiles such a rule would read (pinned), while the rule itself
+is the caller's and is "parity unpinned".
 """

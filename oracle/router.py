@@ -20,6 +20,17 @@ Readings (the pages leave these open):
      The output order is the selection order.
   R9 The "16th/17th gap" of a token is sigmoid(z_(k)) - sigmoid(z_(k+1)) in fp64
      (z_(i) is the i-th largest logit); it is +inf when k == E.
+  R23 Quantile Balancing inputs.  The router rows of the component tables set each
+     expert's selection bias every step from "a quantile of routing margins", and
+     "Kimi K3, previewed" (embedl blog), "Stable LatentMoE" section, has the
+     allocation derived from router-score quantiles.  The rule itself is not
+     published.  Reading of what it reads: the routing margin of expert e for token
+     t is m[t, e] = key[t, e] - key_(k)(t), the distance of the expert's selection
+     key (z, or z + b in the select-only mode) from the token's k-th largest key,
+     the threshold of its top-k; selected experts have m >= 0.  The per-expert
+     quantile at level q over the step's T tokens is the order statistic of rank
+     j = clamp(ceil(q T), 1, T) of m[:, e] (the inverse of the empirical CDF).
+     Keys and margins are formed in the precision of the z passed in.
   R20 Select-only bias (second mode).  The same rows call b a per-expert
      *selection* bias, and the raw config of "Kimi K3" (llm-atlas) has
      topk_method noaux_tc.  The plainest reading of both: experts are chosen
@@ -90,3 +101,43 @@ def route(z, k, select_bias=None):
     else:
         gap = np.full(T, np.inf)
     return idx, w, gap
+
+
+def routing_margins(z, k, select_bias=None):
+    """m[t, e] = key[t, e] - key_(k)(t), the k-th largest key of token t (R23).
+
+    key = z, or z + select_bias in the select-only mode (R20); both the key and the
+    difference are formed in the precision of z (fp32 logits give fp32 margins).
+    Returns an array shaped like z.
+    """
+    z_in = np.asarray(z)
+    key = z_in if select_bias is None else z_in + np.asarray(select_bias, dtype=z_in.dtype)[None, :]
+    T, E = key.shape
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    theta = -np.sort(-key, axis=1)[:, k - 1]          # k-th largest key of each token
+    return (key - theta[:, None]).astype(z_in.dtype)
+
+
+def quantile_rank(q, T):
+    """Rank j (1-based) of the order statistic that is the level-q quantile of T values:
+    clamp(ceil(q T), 1, T), computed in fp64 (R23)."""
+    j = int(np.ceil(np.float64(q) * np.float64(T)))
+    return min(max(j, 1), T)
+
+
+def margin_quantiles(m, levels):
+    """Per-expert quantiles of the margins m [T, E] at the given levels (R23).
+
+    Returns [len(levels), E] in m's dtype: entry (i, e) is the order statistic of rank
+    quantile_rank(levels[i], T) of the column m[:, e].
+    """
+    m = np.asarray(m)
+    T, E = m.shape
+    if T == 0:
+        raise ValueError("need T >= 1")
+    col_sorted = np.sort(m, axis=0)                     # ascending, per expert
+    out = np.empty((len(levels), E), dtype=m.dtype)
+    for i, q in enumerate(levels):
+        out[i] = col_sorted[quantile_rank(q, T) - 1]
+    return out

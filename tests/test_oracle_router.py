@@ -162,3 +162,77 @@ def test_select_only_key_in_fp32_when_given_fp32():
     idx64, _, _ = router.route(z2.astype(np.float64), 1, select_bias=b2.astype(np.float64))
     assert idx64[0, 0] == 1                       # in fp64 the key of expert 1 is larger
     assert router.route(z, 1, select_bias=b)[0][0, 0] == 1
+
+
+# ------------------------------------------------------------------ Quantile Balancing inputs (R23)
+def test_routing_margins_hand_computed():
+    # k = 2: the threshold is the 2nd largest logit (2.0)
+    z = np.array([[3.0, 1.0, 2.0, 0.0]])
+    assert np.array_equal(router.routing_margins(z, 2), [[1.0, -1.0, 0.0, -2.0]])
+    # select-only: the key is z + b; with z = 0 the margins are b minus its 2nd largest value
+    b = np.array([1.0, 3.0, 2.0, 0.0])
+    assert np.array_equal(router.routing_margins(np.zeros((1, 4)), 2, select_bias=b), [[-1.0, 1.0, 0.0, -2.0]])
+    # k = E: every expert is selected, the threshold is the smallest key
+    assert np.array_equal(router.routing_margins(z, 4), [[3.0, 1.0, 2.0, 0.0]])
+
+
+def test_routing_margins_agree_with_the_selection():
+    """With distinct keys, exactly the selected experts have m >= 0, the k-th selected one
+    has m == 0, and m keeps the order of the keys within a token."""
+    g = np.random.default_rng(4)
+    for T, E, k in ((50, 32, 4), (20, 896, 16), (9, 5, 5)):
+        z = g.standard_normal((T, E))
+        m = router.routing_margins(z, k)
+        idx = router.topk_select(z, k)
+        sel = np.zeros((T, E), bool)
+        np.put_along_axis(sel, idx.astype(np.int64), True, axis=1)
+        assert np.array_equal(m >= 0, sel)
+        assert np.all(m[np.arange(T), idx[:, k - 1]] == 0.0)
+        assert np.array_equal(np.argsort(-m, axis=1, kind="stable"), np.argsort(-z, axis=1, kind="stable"))
+
+
+def test_routing_margins_in_fp32_for_fp32_logits():
+    """fp32 logits give fp32 margins: each one is the correctly rounded fp32 difference,
+    which is what an fp32 kernel computes."""
+    g = np.random.default_rng(5)
+    z = g.standard_normal((30, 64)).astype(np.float32)
+    b = (g.standard_normal(64) * 0.1).astype(np.float32)
+    m = router.routing_margins(z, 6, select_bias=b)
+    assert m.dtype == np.float32
+    key = (z + b).astype(np.float64)                   # fp32 sums, held exactly in fp64
+    for t in range(30):
+        theta = sorted(key[t], reverse=True)[5]
+        for e in range(64):
+            assert m[t, e] == np.float32(key[t, e] - theta)   # exact difference, rounded once
+
+
+def test_quantile_rank_and_quantiles_hand_computed():
+    col = np.array([[5.0], [1.0], [3.0], [2.0]])       # sorted: 1, 2, 3, 5
+    levels = [0.0, 0.25, 0.26, 0.5, 0.75, 0.99, 1.0]
+    assert [router.quantile_rank(q, 4) for q in levels] == [1, 1, 2, 2, 3, 4, 4]
+    assert np.array_equal(router.margin_quantiles(col, levels)[:, 0], [1, 1, 2, 2, 3, 5, 5])
+
+
+def test_margin_quantiles_are_numpys_inverted_cdf_quantiles():
+    """The level-q quantile (R23) is numpy's "inverted_cdf" method (the inverse of the
+    empirical distribution function), column by column."""
+    g = np.random.default_rng(6)
+    m = g.standard_normal((257, 40))
+    levels = [0.0, 0.01, 1 / 3, 0.5, 0.9, 1 - 16 / 896, 1.0]
+    got = router.margin_quantiles(m, levels)
+    for i, q in enumerate(levels):
+        assert np.array_equal(got[i], np.quantile(m, q, axis=0, method="inverted_cdf"))
+
+
+def test_margin_quantiles_planted_threshold_mistake_is_caught():
+    """Taking the (k+1)-th key as the threshold (a plausible slip) breaks the pin that
+    selected experts are exactly those with m >= 0."""
+    g = np.random.default_rng(7)
+    z = g.standard_normal((40, 32))
+    k = 4
+    wrong = z - (-np.sort(-z, axis=1))[:, k][:, None]
+    idx = router.topk_select(z, k)
+    sel = np.zeros(z.shape, bool)
+    np.put_along_axis(sel, idx.astype(np.int64), True, axis=1)
+    assert not np.array_equal(wrong >= 0, sel)
+    assert np.array_equal(router.routing_margins(z, k) >= 0, sel)
