@@ -3,7 +3,9 @@
 One step = the whole hot path on one batch: moe_route (router GEMM, sigmoid top-k) and
 moe_forward (grouping, MXFP8 quantise, gate/up grouped GEMM + GLU + requant, down grouped
 GEMM, shared expert, combine), inputs resident in HBM.  Default workload: Kimi-K3 prefill,
-T=8192 tokens, d=7168, 896 experts, top-16, I=3072, one bf16 shared expert (I=3072).
+T=8192 tokens, d=7168, 896 experts, top-16, I=3072, one bf16 shared expert (I=3072).  The
+default line also carries a `decode` object: the Kimi-K3 decode step (T=64, seed 1, same
+shapes) timed the same way, with its fraction of the measured HBM bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -13,6 +15,7 @@ Multi-GPU: token batches are independent, so N ranks run N replicas of the workl
 (rank 0 only) and extrapolates to the full batch.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -27,11 +30,16 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s at K3 shape (T=8192); % FP4 tensor peak, decode % HBM BW"
 UNIT = "tokens/s"
 
-# DRAM bytes (read + write) of one launch of the routed gate/up GEMM on the T=8192
-# workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` of this
-# kernel version (profiles/dram_gemm_k3_prefill_t8192.md).  None whenever the kernel
-# has changed since that capture.
-GATE_UP_TRAFFIC_BYTES = {8192: 24049482240 + 408422400}
+# The GEMM sources whose hash keys a recorded DRAM-traffic figure.
+GEMM_SOURCES = ("gemm.cuh", "ptx.cuh", "tiling.cuh")
+# DRAM bytes (read + write) of one launch of the routed gate/up GEMM, from an ncu capture
+# (`--metrics dram__bytes_read.sum,dram__bytes_write.sum`, one pass) of the kernel built
+# from the GEMM sources with the given hash.  A figure whose hash no longer matches the
+# sources is not reported.
+GATE_UP_TRAFFIC = {
+    ("k3_prefill_t8192", 8192): {"bytes": 24049482240 + 408422400, "sha16": "5e4085c75463c969",
+                                  "how": "timed-step launch of the full T=8192 workload"},
+}
 
 
 def parse():
@@ -44,6 +52,8 @@ def parse():
     ap.add_argument("--T", type=int, default=None, help="override the token count")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode (T=64) measurement that the default workload adds")
     ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 160],
                     help="grouped-GEMM token rows per tile (0 = the library's per-call choice)")
     return ap.parse_args()
@@ -213,15 +223,53 @@ def setup(wl, T, device):
     return x, W_r, bias, plan, ex, sh
 
 
-def run_ours(args, rank, world, local_rank):
+def source_sha16(*names):
+    """First 16 hex digits of the sha256 of the named CUDA sources of the package."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "block_scaled_moe_sigmoid_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def peaks_from_file():
+    peaks = {}
+    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk_path):
+        peaks = json.load(open(pk_path))
+    if peaks.get("bf16_tflops_sustained"):
+        bf16, peak_src = peaks["bf16_tflops_sustained"], "measured"
+    else:
+        bf16, peak_src = 1400.0, "fallback"
+    hbm, hbm_src = (peaks["hbm_gbs"], "measured") if peaks.get("hbm_gbs") else (6650.0, "fallback")
+    return bf16, peak_src, hbm, hbm_src
+
+
+def count_launches(api, plan, stages):
+    """Kernels launched by the recorded stage instances (profiled pass)."""
+    launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_ROUTER_SPLIT) > 1:
+        launches += stages["router_gemm"][1]   # the K-split partial sum
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1:
+        launches += stages["shared_gate_up"][1]
+    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT_DOWN) > 1:
+        launches += stages["shared_down"][1]
+    return launches
+
+
+def measure(args, wl, T, world, local_rank, e2e_on):
+    """Time `args.steps` steps of the workload (route + forward) on resident inputs.
+
+    1. Timed pass: CUDA events on the launching stream around the K steps, stage profiler
+       off, barrier + synchronize on both sides, max over ranks.
+    2. Profiled pass: the same K steps again with the per-stage event profiler on, for the
+       per-kernel launch times (roofline) and the launch count.
+    3. Optionally the end-to-end pass with host buffers."""
     import torch
     import torch.distributed as dist
 
-    from block_scaled_moe_sigmoid_b200 import api, synth
-    wl = synth.WORKLOADS[args.workload]
-    T = args.T or (wl.sweep[-1] if wl.sweep else wl.T)
+    from block_scaled_moe_sigmoid_b200 import api
     dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
     x, W_r, bias, plan, ex, sh = setup(wl, T, "cuda")
     api.moe_plan_set_option(plan.handle, api.MOE_OPT_TILE_N, args.tile_n)
     idx = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
@@ -246,10 +294,9 @@ def run_ours(args, rank, world, local_rank):
     def max_over_ranks(v):
         return max_over_ranks_(v, world, dev)
 
-    # ---- timed region (device time, CUDA events on the launching stream)
+    # ---- 1. timed pass (device time, CUDA events on the launching stream)
     clocks = ClockSampler(local_rank)
     clocks.start()
-    api.moe_plan_set_profiling(plan.handle, True)
     barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -260,27 +307,31 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
-    stages = api.moe_plan_stage_ms(plan.handle)
-    api.moe_plan_set_profiling(plan.handle, False)
     clk = clocks.stop()
     code, bits = plan.check()
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} in the timed region")
-    launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
-    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_ROUTER_SPLIT) > 1:
-        launches += stages["router_gemm"][1]   # the K-split partial sum
-    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1:
-        launches += stages["shared_gate_up"][1]
-    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT_DOWN) > 1:
-        launches += stages["shared_down"][1]
 
-    # ---- end to end through the public API with host buffers
+    # ---- 2. profiled pass: per-stage launch times and the launch count
+    api.moe_plan_set_profiling(plan.handle, True)
+    barrier()
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        one_step()
+    torch.cuda.synchronize()
+    barrier()
+    stages = api.moe_plan_stage_ms(plan.handle)
+    api.moe_plan_set_profiling(plan.handle, False)
+    launches = count_launches(api, plan, stages)
+
+    # ---- 3. end to end through the public API with host buffers
     # Every step copies its input x from pinned host memory and its output y back, inside
     # the timed region.  The copies run on their own streams, double-buffered, so step i's
     # output copy and step i+1's input copy overlap the compute of the neighbouring steps,
-    # as a serving loop would run them.  Each step's compute waits for its own input copy.
+    # as a serving loop would run them.  Each step's compute waits for its own input copy,
+    # and the first input copy of the timed region waits for its start event.
     e2e = None
-    if not args.no_e2e:
+    if e2e_on:
         x_host = x.cpu().pin_memory()
         y_host = [torch.empty((T, wl.d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]
@@ -288,9 +339,11 @@ def run_ours(args, rank, world, local_rank):
         h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
         ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("h2d", "comp", "d2h")}
 
-        def e2e_step(i):
+        def e2e_step(i, start=None):
             b = i % 2
             with torch.cuda.stream(h2d):
+                if start is not None:
+                    h2d.wait_event(start)                # nothing of the step before the window
                 if i >= 2:
                     h2d.wait_event(ev["comp"][b])        # step i-2 is done with x_dev[b]
                 x_dev[b].copy_(x_host, non_blocking=True)
@@ -313,7 +366,7 @@ def run_ours(args, rank, world, local_rank):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(args.steps):
-            e2e_step(i)
+            e2e_step(i, start=e0 if i == 0 else None)
         for b in range(2):
             stream.wait_event(ev["d2h"][b])              # the last outputs are on the host
         e1.record(stream)
@@ -325,34 +378,32 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": y.numel() * y.element_size(),
                "overlap": "copies on their own streams, double-buffered across steps"}
 
-    # ---- roofline of the dominant kernel (routed gate/up GEMM)
-    # Its bound is the slower of two terms: the block-scaled MMAs at the tensor pipe's rate
-    # for MXFP4 x MXFP8 operands (kind::mxf8f6f4 issues at the FP8 rate, twice bf16), and
-    # the algorithmic HBM bytes (the touched experts' codes and scales, the MXFP8 token rows
-    # read once, the MXFP8 GLU output written once) at the measured copy bandwidth.
-    peaks = {}
-    pk_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(pk_path):
-        peaks = json.load(open(pk_path))
-    if peaks.get("bf16_tflops_sustained"):
-        bf16, peak_src = peaks["bf16_tflops_sustained"], "measured"
-    else:
-        bf16, peak_src = 1400.0, "fallback"
-    hbm, hbm_src = (peaks["hbm_gbs"], "measured") if peaks.get("hbm_gbs") else (6650.0, "fallback")
     touched = int(torch.unique(idx).numel())
-    # per-expert load of the timed routing (assignments per expert), summarised
     load = torch.bincount(idx.reshape(-1).long(), minlength=wl.E).cpu()
-    ls = torch.sort(load, descending=True).values
-    expert_load = {"mean": float(load.float().mean()), "max": int(ls[0]), "min": int(ls[-1]),
-                   "p50": int(ls[wl.E // 2]), "p90": int(ls[wl.E // 10]), "zero_experts": int((load == 0).sum()),
-                   "top8": [int(v) for v in ls[:8]],
-                   "share_of_top_1pct": float(ls[:max(1, wl.E // 100)].sum()) / max(1, int(load.sum()))}
-    gu_ms, gu_n = stages["gate_up_glu"]
+    tile_rows = api.moe_plan_get_option(plan.handle, api.MOE_OPT_TILE_N)
+    res = {"ms": ms, "stages": stages, "launches": launches, "clocks": clk, "e2e": e2e,
+           "touched": touched, "load": load, "tile_rows": tile_rows}
+    # the host copies the CPU baseline needs (the oracle reads the same draws)
+    res["data"] = (x, W_r, bias)
+    del plan, ex, sh, y, idx, w
+    torch.cuda.empty_cache()
+    return res
+
+
+def gate_up_roofline(wl, T, m, traffic):
+    """Roofline object of the routed gate/up GEMM, the dominant kernel.
+
+    Its bound is the slower of two terms: the block-scaled MMAs at the tensor pipe's rate
+    for MXFP4 x MXFP8 operands (kind::mxf8f6f4 issues at the FP8 rate, twice bf16), and the
+    algorithmic HBM bytes (the touched experts' codes and scales, the MXFP8 token rows read
+    once, the MXFP8 GLU output written once) at the measured copy bandwidth."""
+    bf16, peak_src, hbm, hbm_src = peaks_from_file()
+    gu_ms, gu_n = m["stages"]["gate_up_glu"]
     t_launch = gu_ms / gu_n / 1e3 if gu_n else None
     A = T * wl.k
     de = wl.d_expert                                           # expert input width (d, or d_latent)
     flops = 2.0 * A * de * (2 * wl.I)
-    gu_bytes = (touched * 2 * wl.I * de * 17 / 32             # E2M1 codes + E8M0 scales
+    gu_bytes = (m["touched"] * 2 * wl.I * de * 17 / 32        # E2M1 codes + E8M0 scales
                 + A * de * 33 / 32 + A * wl.I * 33 / 32)       # MXFP8 rows in, GLU rows out
     tc_peak = 2.0 * bf16
     tensor_bound = flops / tc_peak / 1e12 >= gu_bytes / hbm / 1e9
@@ -362,23 +413,87 @@ def run_ours(args, rank, world, local_rank):
     else:
         achieved = gu_bytes / t_launch / 1e9 if t_launch else None
         peak, unit = hbm, "GB/s"
-    traffic = GATE_UP_TRAFFIC_BYTES.get(T) if args.workload == "k3_prefill_t8192" else None
-    roofline = {"kernel": "gemm_kernel<KIND_MX, EPI_GLU_MX8> (routed gate/up + SiLU-GLU + MXFP8 requant)",
-                "bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak if achieved else None, "traffic": traffic,
-                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-                "peak_note": (f"tensor: FP8-rate pipe = 2 x {peak_src} sustained bf16 GEMM "
-                              f"(kind::mxf8f6f4 issues at the FP8 rate); hbm: {hbm_src} copy bandwidth"),
-                "ms_per_launch": gu_ms / gu_n if gu_n else None,
-                "flops_per_launch": flops, "algorithmic_bytes_per_launch": gu_bytes,
-                "touched_experts": touched,
-                "tflops_per_launch": flops / t_launch / 1e12 if t_launch else None,
-                "frac_of_nominal_fp4_rate": (flops / t_launch / 1e12 / (4.0 * bf16)) if t_launch else None,
-                "fp4_note": "FP4-rate MMAs (kind::mxf4) need both operands in E2M1; MXFP8 "
-                            "activations run at the FP8 rate, so the FP4 figure is context"}
-    w_bytes = (touched * 3 * de * wl.I * 17 / 32 + 3 * wl.d * wl.I_shared * 2
-               + wl.d * wl.E * 4 + 2 * wl.d * wl.d_latent * 2)
-    stage_ms = {k: round(v[0] / max(v[1], 1), 4) for k, v in stages.items()}
+    return {"kernel": "gemm_kernel<KIND_MX, EPI_GLU_MX8> (routed gate/up + SiLU-GLU + MXFP8 requant)",
+            "bound": "tensor" if tensor_bound else "hbm", "achieved": achieved, "peak": peak,
+            "unit": unit, "frac": achieved / peak if achieved else None,
+            "traffic": traffic["bytes"] if traffic else None,
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+            "traffic_source": traffic["source"] if traffic else
+            "none recorded for this kernel source and workload",
+            "peak_note": (f"tensor: FP8-rate pipe = 2 x {peak_src} sustained bf16 GEMM "
+                          f"(kind::mxf8f6f4 issues at the FP8 rate); hbm: {hbm_src} copy bandwidth"),
+            "ms_per_launch": gu_ms / gu_n if gu_n else None,
+            "launch_time_source": "per-stage CUDA events on the launching stream, profiled pass "
+                                  "of the same steps",
+            "flops_per_launch": flops, "algorithmic_bytes_per_launch": gu_bytes,
+            "hbm_frac_of_algorithmic_bytes": (gu_bytes / t_launch / 1e9 / hbm) if t_launch else None,
+            "touched_experts": m["touched"],
+            "tflops_per_launch": flops / t_launch / 1e12 if t_launch else None,
+            "frac_of_nominal_fp4_rate": (flops / t_launch / 1e12 / (4.0 * bf16)) if t_launch else None,
+            "fp4_note": "FP4-rate MMAs (kind::mxf4) need both operands in E2M1; MXFP8 "
+                        "activations run at the FP8 rate, so the FP4 figure is context"}
+
+
+def weight_bytes(wl, touched):
+    """Touched experts' MXFP4 weights + bf16 shared expert + fp32 router matrix (+ latent
+    projections) streamed per step."""
+    de = wl.d_expert
+    return (touched * 3 * de * wl.I * 17 / 32 + 3 * wl.d * wl.I_shared * 2
+            + wl.d * wl.E * 4 + 2 * wl.d * wl.d_latent * 2)
+
+
+def traffic_record(workload, T):
+    """The recorded ncu DRAM bytes of one gate/up launch, when they were captured on the
+    current GEMM source; None otherwise (a stale figure is not reported)."""
+    rec = GATE_UP_TRAFFIC.get((workload, T))
+    if not rec:
+        return None
+    sha = source_sha16(*GEMM_SOURCES)
+    if rec["sha16"] != sha:
+        return None
+    return {"bytes": rec["bytes"],
+            "source": f"ncu capture of this gate/up kernel (csrc sha {sha}), {rec['how']}"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from block_scaled_moe_sigmoid_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    T = args.T or (wl.sweep[-1] if wl.sweep else wl.T)
+    torch.cuda.set_device(torch.device("cuda", local_rank))
+    m = measure(args, wl, T, world, local_rank, e2e_on=not args.no_e2e)
+    ms = m["ms"]
+    _, _, hbm, _ = peaks_from_file()
+    roofline = gate_up_roofline(wl, T, m, traffic_record(args.workload, T))
+    w_bytes = weight_bytes(wl, m["touched"])
+    stage_ms = {k: round(v[0] / max(v[1], 1), 4) for k, v in m["stages"].items()}
+    load = m["load"]
+    ls = torch.sort(load, descending=True).values
+    expert_load = {"mean": float(load.float().mean()), "max": int(ls[0]), "min": int(ls[-1]),
+                   "p50": int(ls[wl.E // 2]), "p90": int(ls[wl.E // 10]), "zero_experts": int((load == 0).sum()),
+                   "top8": [int(v) for v in ls[:8]],
+                   "share_of_top_1pct": float(ls[:max(1, wl.E // 100)].sum()) / max(1, int(load.sum()))}
+
+    # ---- the decode half of the metric: the Kimi-K3 decode step (T=64), same shapes
+    decode = None
+    if args.workload == "k3_prefill_t8192" and not args.no_decode:
+        dwl = synth.WORKLOADS["k3_decode_t64"]
+        dm = measure(args, dwl, dwl.T, world, local_rank, e2e_on=False)
+        d_ms = dm["ms"] / args.steps
+        d_bytes = weight_bytes(dwl, dm["touched"])
+        d_roof = gate_up_roofline(dwl, dwl.T, dm, None)
+        decode = {"workload": dwl.name, "T": dwl.T, "seed": dwl.seed, "ms_per_step": d_ms,
+                  "value": world * dwl.T / (d_ms / 1e3), "unit": UNIT,
+                  "touched_experts": dm["touched"], "weight_bytes_per_step": d_bytes,
+                  "frac_hbm": d_bytes / (d_ms / 1e3) / 1e9 / hbm,
+                  "gate_up_frac_hbm": d_roof["hbm_frac_of_algorithmic_bytes"],
+                  "gate_up_ms_per_launch": d_roof["ms_per_launch"],
+                  "stage_ms_per_launch": {k: round(v[0] / max(v[1], 1), 4) for k, v in dm["stages"].items()},
+                  "gpu_launches": dm["launches"], "clocks": dm["clocks"],
+                  "note": "frac_hbm = touched experts' MXFP4 weights + shared expert + router "
+                          "matrix per step over the step's device time, against the measured "
+                          "copy bandwidth; 20 GB+ of weights per step, so no L2 reuse between steps"}
 
     out = None
     if rank == 0:
@@ -392,18 +507,20 @@ def run_ours(args, rank, world, local_rank):
                        "k": wl.k, "I": wl.I,
                        "I_shared": wl.I_shared, "seed": wl.seed, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2: every step streams "
-                             f"{w_bytes / 1e9:.1f} GB of weights ({touched} touched experts)"},
+                             f"{w_bytes / 1e9:.1f} GB of weights ({m['touched']} touched experts)"},
             "roofline": roofline,
-            "gemm_tile_rows": api.moe_plan_get_option(plan.handle, api.MOE_OPT_TILE_N),
+            "decode": decode,
+            "gemm_tile_rows": m["tile_rows"],
             "expert_load": expert_load,
-            "hbm_view": {"weight_bytes_per_step": w_bytes, "touched_experts": touched,
+            "hbm_view": {"weight_bytes_per_step": w_bytes, "touched_experts": m["touched"],
                          "achieved_gbs": w_bytes / (ms / args.steps / 1e3) / 1e9,
                          "peak_gbs": hbm, "frac": w_bytes / (ms / args.steps / 1e3) / 1e9 / hbm,
                          "note": "touched experts' MXFP4 weights + bf16 shared expert + fp32 "
                                  "router matrix per step, over the whole step's time"},
             "stage_ms_per_launch": stage_ms,
-            "clocks": clk, "e2e": e2e, "gpu_launches": launches,
+            "clocks": m["clocks"], "e2e": m["e2e"], "gpu_launches": m["launches"],
         }
+    x, W_r, bias = m["data"]
     return out, (x, W_r, bias, wl, T)
 
 

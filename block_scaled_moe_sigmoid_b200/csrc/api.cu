@@ -888,25 +888,55 @@ moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes
 static constexpr size_t kNoAllocScratchBytes = 256 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the scratch array on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device (with
-// that device current) and cached.
+// Device address of the scratch array in the current context.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up with the device current
+// (cudaGetSymbolAddress, return code checked) once per device and context, and cached.  The
+// cache is keyed on the context's unique id (cuCtxGetId): after cudaDeviceReset, or under
+// another context on the same device, the address is looked up again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = (CtxGetCurrentFn)p;
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (CtxGetIdFn)p;
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 static void* noalloc_scratch(moe_status_t* st) {
   static std::mutex mu;
   static void* addr[64] = {};
+  static unsigned long long ctx_of[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     *st = MOE_ERR_CUDA;
     return nullptr;
   }
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !have_id || ctx_of[dev] != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       *st = MOE_ERR_CUDA;
       return nullptr;
     }
     addr[dev] = p;
+    ctx_of[dev] = have_id ? id : 0;
   }
   return addr[dev];
 }

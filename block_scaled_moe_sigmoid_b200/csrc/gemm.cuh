@@ -231,6 +231,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* drain_sf = drain_bar + 1;
   uint32_t* tmem_holder = (uint32_t*)(drain_sf + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
+  // Fill counters for the abort cleanup: [0] weight producer, [1] token producer, [2] scale
+  // warp (sf_full fills consumed = full-barrier arrivals made), [3] MMA (fills consumed).
+  int* fills = (int*)(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -248,6 +251,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(smem_u32(drain_bar), 1);
     mbar_init(smem_u32(drain_sf), 1);
     *abort_flag = 0;
+    for (int r = 0; r < 4; ++r) fills[r] = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
   }
@@ -290,6 +294,7 @@ __global__ void __launch_bounds__(384, 1)
     };
     for (int i = 0; i < args.pf_dist; ++i) prefetch_one();
     bool ok = true;
+    int nfill = 0;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
@@ -320,10 +325,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
+        ++nfill;
         prefetch_one();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
+    if (lane == 0) fills[0] = nfill;
   } else if (warp == 10) {
     // ------------------------------------------------------------- producer: token rows
     // One TMA box of the tile's rows (box height 32 * nB, nB = ceil(n_mma / 32)) and
@@ -332,6 +339,7 @@ __global__ void __launch_bounds__(384, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int nfill = 0;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
@@ -358,9 +366,11 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         __syncwarp();
+        ++nfill;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
+    if (lane == 0) fills[1] = nfill;
   } else if (warp == 11) {
     // ------------------------------------------------------------- scale factors -> TMEM
     // tcgen05.cp of each stage's scale atoms into that stage's TMEM buffer, off the MMA
@@ -374,6 +384,7 @@ __global__ void __launch_bounds__(384, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int nfill = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         TileInfo ti;
         gemm_decode_tile(args, BN_MAX, t, ti);
@@ -382,6 +393,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int kt = ti.kb; kt < ti.ke; ++kt) {
           ok = mbar_wait(smem_u32(sf_full + stage), phase, args.status, abort_flag);
           if (!ok) break;
+          ++nfill;
           tc_fence_after();
           const uint64_t sfa_desc = sf_desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
           const uint64_t sfb_desc = sfa_desc + (uint64_t)(C::SFA_BYTES >> 4);
@@ -394,8 +406,10 @@ __global__ void __launch_bounds__(384, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // every scale copy this warp issued lands before TMEM is released
       tc_commit(smem_u32(drain_sf));
-      mbar_wait(smem_u32(drain_sf), 0, args.status, abort_flag);
+      mbar_wait_drain(smem_u32(drain_sf), 0);
+      fills[2] = nfill;
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -406,6 +420,7 @@ __global__ void __launch_bounds__(384, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      int nfill = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         TileInfo ti;
         gemm_decode_tile(args, BN_MAX, t, ti);
@@ -450,7 +465,11 @@ __global__ void __launch_bounds__(384, 1)
           const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
-          if (ok && two) ok = mbar_wait(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
+          if (ok) ++nfill;
+          if (ok && two) {
+            ok = mbar_wait(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
+            if (ok) ++nfill;
+          }
           if (!ok) break;
           tc_fence_after();
           issue_stage(stage, kt > ti.kb ? 1u : 0u);
@@ -471,7 +490,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       // make sure every MMA this thread issued has finished before TMEM is released
       tc_commit(smem_u32(drain_bar));
-      mbar_wait(smem_u32(drain_bar), 0, args.status, abort_flag);
+      mbar_wait_drain(smem_u32(drain_bar), 0);
+      fills[3] = nfill;
     }
     __syncwarp();
   } else {
@@ -601,8 +621,13 @@ __global__ void __launch_bounds__(384, 1)
 
   __syncthreads();
   if (*abort_flag) {
-    // let any bulk copies still in flight land before the CTA's shared memory goes away
-    __nanosleep(100000);
+    // A role gave up: let every copy still in flight into this CTA's shared memory land
+    // (supplying the arrivals of the roles that stopped early) before the CTA exits.
+    if (threadIdx.x == 0) {
+      drain_ring(full_bar, STAGES, fills, KIND == KIND_MX ? 3 : 2, fills[3]);
+      if constexpr (KIND == KIND_MX) drain_ring(sf_full, STAGES, fills, 2, fills[2]);
+    }
+    __syncthreads();
   }
   if (warp == 1) {
     tc_fence_after();

@@ -75,6 +75,40 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+#ifndef MOE_DRAIN_LIMIT_NS
+#define MOE_DRAIN_LIMIT_NS 20000000ull  // 20 ms
+#endif
+
+// Bounded wait used on the way out of a CTA that gave up: it ignores the abort flag, so
+// that copies and tensor-core operations the CTA already issued can finish before its
+// shared memory and TMEM are released.  Returns false after MOE_DRAIN_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > MOE_DRAIN_LIMIT_NS) return false;
+  return true;
+}
+
+// Abort cleanup of a ring of `stages` mbarriers that several roles fill in turn.  Fill f
+// uses barrier f % stages in phase (f / stages) & 1; role r arrived on fills [0, arrived[r])
+// (a producer's arrival is its arrive.expect_tx, issued together with its copies), and the
+// consumer waited on fills [0, consumed).  Every fill in [consumed, max arrived) still has
+// copies in flight or arrivals missing: the missing arrivals are supplied here, so each
+// phase completes as soon as its bytes have landed, and that is waited for (bounded).
+// One thread, after every role has stopped issuing.
+__device__ __forceinline__ void drain_ring(uint64_t* bars, int stages, const int* arrived, int roles,
+                                           int consumed) {
+  int last = consumed;
+  for (int r = 0; r < roles; ++r) last = max(last, arrived[r]);
+  for (int f = consumed; f < last; ++f) {
+    const uint32_t bar = smem_u32(bars + f % stages);
+    for (int r = 0; r < roles; ++r)
+      if (arrived[r] <= f) mbar_arrive(bar);
+    mbar_wait_drain(bar, (uint32_t)(f / stages) & 1u);
+  }
+}
+
 // ---------------------------------------------------------------- TMA / async copies
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int x, int y, uint64_t policy) {

@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain_bar = pempty + 2;
   uint32_t* tmem_holder = (uint32_t*)(drain_bar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
+  int* fills = (int*)(tmem_holder + 2);   // abort cleanup: [0] loads armed, [1] loads consumed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tok_tiles = (args.T + RBN - 1) / RBN;
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
+    fills[0] = fills[1] = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
@@ -108,6 +110,7 @@ __global__ void __launch_bounds__(320, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int nfill = 0;
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       const RouterTile rt = router_tile(args, RBN, t);
       const int mt = rt.mt, row0 = rt.row0;
@@ -128,9 +131,11 @@ __global__ void __launch_bounds__(320, 1)
           for (int i = 0; i < nB; ++i) tma_load_2d(smem_u32(sB + i * 4096), &tmB, fb, c * 64, row0 + 32 * i, pol);
         }
         __syncwarp();
+        ++nfill;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
+    if (lane == 0) fills[0] = nfill;
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA: one chain per stage
     if (lane == 0) {
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t phase = 0;
       uint32_t g = 0;  // chain counter across tiles: buffer g & 1, phase (g >> 1) & 1
       bool ok = true;
+      int nfill = 0;
       const uint64_t desc0 = smem_desc(smem_u32(smem), 16, 1024, 2);  // stage 0, plane 0
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const RouterTile rt = router_tile(args, RBN, t);
@@ -150,6 +156,7 @@ __global__ void __launch_bounds__(320, 1)
           if (!ok) break;
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (!ok) break;
+          ++nfill;
           tc_fence_after();
           const uint64_t a_desc = desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
           const uint64_t b_desc = a_desc + (uint64_t)(C::A_BYTES >> 4);
@@ -165,8 +172,10 @@ __global__ void __launch_bounds__(320, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // every MMA this thread issued finishes before TMEM is released
       tc_commit(smem_u32(drain_bar));
-      mbar_wait(smem_u32(drain_bar), 0, args.status, abort_flag);
+      mbar_wait_drain(smem_u32(drain_bar), 0);
+      fills[1] = nfill;
     }
     __syncwarp();
   } else {
@@ -225,7 +234,11 @@ __global__ void __launch_bounds__(320, 1)
   }
 
   __syncthreads();
-  if (*abort_flag) __nanosleep(100000);
+  if (*abort_flag) {
+    // a role gave up: the loads already issued land before the CTA exits
+    if (threadIdx.x == 0) drain_ring(full_bar, STAGES, fills, 1, fills[1]);
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);

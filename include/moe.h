@@ -129,6 +129,10 @@ moe_status_t moe_quant_mxfp8(const void* x_bf16, int rows, int cols, uint8_t* q_
                              uint8_t* scale_e8m0, void* stream);
 
 /* ---- a2/a3: router --------------------------------------------------------------------
+ * Source: "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, row "Sigmoid router
+ * with Quantile Balancing" (sigmoid scores pick 16 of 896 experts); "Kimi K3" (llm-atlas),
+ * raw config fields moe_router_activation_func sigmoid, num_experts_per_token 16,
+ * moe_renormalize true, routed_scaling_factor 1.
  * z = x . W_r + bias (fp32-accurate: W_r is split into three bf16 terms on the tensor
  * cores), s = sigmoid(z); per token the k largest z in descending order (lower expert
  * index on ties) and w_j = s_j / sum of the selected s.  With MOE_BIAS_SELECT_ONLY the
@@ -162,7 +166,8 @@ moe_status_t moe_permute(moe_plan_t plan, const int32_t* idx, int T, int32_t* co
  * bytes exceed it (e.g. T <= 18432 at E = 896).  All calls share the array, so two calls
  * whose work overlaps on the GPU (different streams, or different host threads) race.
  * The first call on a device looks up the array's device address (with that device
- * current) and caches it; make that first call before any stream capture.
+ * current) and caches it per device and CUDA context (a new context, e.g. after
+ * cudaDeviceReset, gets a fresh lookup); make that first call before any stream capture.
  * Arguments and outputs as moe_permute (device pointers, caller-owned); ids outside
  * [0, E) are skipped and leave inv = -1 (no status is reported). */
 moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int32_t* counts,
@@ -170,6 +175,11 @@ moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int32_
                                  void* stream);
 
 /* ---- a4..a9: the layer ----------------------------------------------------------------
+ * Source: "Kimi K3.1 Pro vs gpt-oss-120b" (archdiff), component table, rows "Stable
+ * LatentMoE routed experts (SiTU-GLU)" and "Shared expert", and its block diagram, which
+ * adds the routed and shared outputs; "Kimi K3" (llm-atlas), Key facts, Dtype row (MXFP4
+ * experts, high-precision shared expert); "Kimi K3, previewed" (embedl blog),
+ * specifications figure caption (MXFP4 weights, MXFP8 activations).
  * y = bf16( shared(x) + sum_j w[t][j] * expert_{idx[t][j]}(x) ), where an expert is
  * down(glu(x Wg^T, x Wu^T)) on MXFP8 x and MXFP4 weights, its GLU output requantised
  * to MXFP8, and shared(x) = bf16(glu(x Wsg^T, x Wsu^T)) Wsd^T in bf16/fp32 (glu: the
