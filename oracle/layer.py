@@ -164,14 +164,23 @@ def moe_layer(x, idx, w, expert_weights, shared=None, tokens=None, act="silu",
         ys, _ = shared_expert(x[rows], *shared, act=act)
     else:
         ys = np.zeros((n, d))
-    acc = ys + np.einsum("nk,nkd->nd", w[rows], o)       # fp64, R16
-    y = mx.bf16_round(acc)
+    y = combine(ys, w[rows], o)
     if want_intermediates:
         inter["o"] = o
         inter["y_shared"] = ys
         inter["xq"], inter["xs"] = xq, xs
         return y, inter
     return y
+
+
+def combine(y_shared, w, o):
+    """y = bf16(y_shared + sum_j w_j o_j), summed in fp64 and rounded once (R16).
+
+    y_shared: [n, d]; w: [n, k] routing weights; o: [n, k, d] expert outputs per slot.
+    """
+    acc = np.asarray(y_shared, np.float64) + np.einsum("nk,nkd->nd", np.asarray(w, np.float64),
+                                                       np.asarray(o, np.float64))
+    return mx.bf16_round(acc)
 
 
 def rms_norm(v, gamma, eps=1e-5):

@@ -168,3 +168,52 @@ def test_bf16_round():
     # a value a hair above the tie rounds up (no double rounding through fp32)
     hair = 1.0 + 2.0 ** -8 + 2.0 ** -40
     assert mx.bf16_round(np.array([hair]))[0] == 1.0 + 2.0 ** -7
+
+
+# ------------------------------------------------------------------ the C restatement (oracle/cmx.c)
+def test_c_quantiser_matches_the_numpy_definition():
+    """oracle/cmx.c restates quantize_mx for fp32 input; it must give the same codes and
+    scales on random data over a wide range of magnitudes, on ties and saturation, and on
+    signed zeros and bf16/fp32 subnormals."""
+    from oracle import cmx
+    g = np.random.default_rng(12)
+    x = (g.standard_normal((64, 512)) * np.logspace(-40, 38, 512)[None, :]).astype(np.float32)
+    x[0] = 0.0
+    x[1, :32] = -0.0
+    x[2, :32] = np.float32(448.0 * 2.0 ** 10)
+    x[3, :32] *= np.float32(1e-38)
+    x[3, 5] = np.float32(2.0 ** -149)                    # fp32 subnormal
+    x[4, :32] = [17.0, 19.0, -17.0, 480.0] * 8           # E4M3 ties and saturation
+    x[5, :32] = [2.5, 5.0, 0.25, 0.75, 1.25, 1.75, -2.5, 7.0] * 4   # E2M1 ties
+    # every E2M1 / E4M3 value times a spread of scales, and the midpoints between them
+    vals = np.concatenate([mx._E2M1_POS, -mx._E2M1_POS, mx._E4M3_POS, -mx._E4M3_POS])
+    mids = (mx._E4M3_POS[1:] + mx._E4M3_POS[:-1]) / 2
+    extra = np.concatenate([vals, mids, -mids])
+    extra = np.resize(extra, (len(extra) + 31) // 32 * 32).reshape(-1, 32)
+    extra = np.concatenate([extra * 2.0 ** s for s in (-20, -3, 0, 5, 30)]).astype(np.float32)
+    for data in (x, extra, g.standard_normal((300, 96)).astype(np.float32) * 0.02):
+        for fmt in ("e2m1", "e4m3"):
+            c1, s1 = cmx.quantize_mx_f32(data, fmt)
+            c0, s0 = mx.quantize_mx(data, fmt)
+            assert np.array_equal(s1, s0), fmt
+            assert np.array_equal(c1, c0), fmt
+
+
+def test_c_quantiser_round_trips_every_code():
+    """Every finite code of both formats, scaled by 2^s: quantising the decoded value gives
+    back the code and the scale (the exhaustive pin of quantize_mx, applied to the C
+    restatement)."""
+    from oracle import cmx
+    for fmt, top in (("e2m1", 8), ("e4m3", 127)):
+        pos = mx._E2M1_POS if fmt == "e2m1" else mx._E4M3_POS
+        for s in (-20, 0, 17):
+            for c in range(1, top):
+                # block: the largest code sets the scale, the tested code sits beside it
+                blk = np.zeros(32)
+                blk[0] = pos[top - 1] * 2.0 ** s
+                blk[1] = pos[c] * 2.0 ** s
+                blk[2] = -pos[c] * 2.0 ** s
+                codes, scales = cmx.quantize_mx_f32(blk[None, :].astype(np.float32), fmt)
+                assert scales[0, 0] == s + 127       # amax = largest value x 2^s: exponent s
+                dec = mx.dequantize_mx(codes, scales, fmt)
+                assert dec[0, 1] == blk[1] and dec[0, 2] == blk[2], (fmt, s, c)
