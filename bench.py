@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode (T=64) measurement that the default workload adds")
-    ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 160],
+    ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 128, 176],
                     help="grouped-GEMM token rows per tile (0 = the library's per-call choice)")
     return ap.parse_args()
 
@@ -248,8 +248,6 @@ def peaks_from_file():
 def count_launches(api, plan, stages):
     """Kernels launched by the recorded stage instances (profiled pass)."""
     launches = sum(cnt * api.STAGE_KERNELS.get(name, 1) for name, (_, cnt) in stages.items())
-    if api.moe_plan_get_option(plan.handle, api.MOE_OPT_ROUTER_SPLIT) > 1:
-        launches += stages["router_gemm"][1]   # the K-split partial sum
     if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT) > 1:
         launches += stages["shared_gate_up"][1]
     if api.moe_plan_get_option(plan.handle, api.MOE_OPT_SHARED_SPLIT_DOWN) > 1:

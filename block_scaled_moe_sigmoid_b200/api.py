@@ -19,6 +19,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_S
 
 # exported symbols and their argument types (ctypes)
 _P, _I, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+# moe_bias_rule_t: (quantiles, n_levels, E, bias, bias_next, stream, user)
+BIAS_RULE = ctypes.CFUNCTYPE(None, _P, _I, _I, _P, _P, _P, _P)
 SIGNATURES = {
     "moe_plan_create": [_I, _I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_P)],
     "moe_plan_workspace_bytes": [_P, ctypes.POINTER(_S)],
@@ -43,12 +45,15 @@ SIGNATURES = {
     "moe_plan_get_option": [_P, _I, ctypes.POINTER(_I)],
     "moe_permute_noalloc": [_P, _I, _I, _I, _P, _P, _P, _P, _P],
     "moe_plan_stage_ms": [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int), _I],
+    "moe_route_margin_quantiles": [_P, _P, _P, _I, ctypes.POINTER(ctypes.c_double), _I, _P, _P],
+    "moe_quantile_balance": [_P, _P, _P, _I, ctypes.POINTER(ctypes.c_double), _I, BIAS_RULE, _P, _P, _P],
 }
+
 
 STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "gate_up_glu",
           "down", "shared_gate_up", "shared_down", "combine", "latent_in", "latent_out"]
-# kernel launches per recorded stage instance (router_gemm: +1 for the partial-sum kernel
-# when moe_plan_get_option(MOE_OPT_ROUTER_SPLIT) > 1)
+# kernel launches per recorded stage instance (the router kernel also sums its K-split
+# partials and selects the top-k, so "topk" records nothing)
 STAGE_KERNELS = {"permute": 3, "quant_scatter": 2, "latent_in": 2, "latent_out": 2}
 
 
@@ -200,6 +205,30 @@ def moe_forward_latent(plan, x, idx, w, latent, experts, shared, y=None, stream=
     _call("moe_forward_latent", plan, _ptr(x), T, _ptr(idx), _ptr(w), ctypes.byref(lat), ctypes.byref(ex),
           ctypes.byref(sh) if sh is not None else None, _ptr(y), _stream(stream))
     return y
+
+
+def moe_route_margin_quantiles(plan, logits, E, levels, select_bias=None, quantiles=None, stream=None):
+    """Per-expert quantiles of the routing margins of logits [T, E] (fp32, device) at the
+    given levels; returns fp32 [len(levels), E] on the device."""
+    T = logits.shape[0]
+    lv = (ctypes.c_double * len(levels))(*levels)
+    if quantiles is None:
+        quantiles = torch.empty((len(levels), E), dtype=torch.float32, device=logits.device)
+    _call("moe_route_margin_quantiles", plan, _ptr(logits), _ptr(select_bias), T, lv, len(levels),
+          _ptr(quantiles), _stream(stream))
+    return quantiles
+
+
+def moe_quantile_balance(plan, logits, bias, levels, rule, bias_next=None, user=None, stream=None):
+    """Margin quantiles of this step, then the caller's rule (a BIAS_RULE callable) writes the
+    next step's bias into bias_next (fp32 [E], device)."""
+    T = logits.shape[0]
+    lv = (ctypes.c_double * len(levels))(*levels)
+    if bias_next is None:
+        bias_next = torch.empty_like(bias)
+    _call("moe_quantile_balance", plan, _ptr(logits), _ptr(bias), T, lv, len(levels), rule, user,
+          _ptr(bias_next), _stream(stream))
+    return bias_next
 
 
 def moe_expert_bytes(d, I, E):

@@ -1,6 +1,8 @@
 // C ABI of the MoE layer (include/moe.h): argument checks, workspace carving, TMA
 // descriptor encoding and the launch sequence.  All arithmetic runs in the kernels of
 // kernels.cuh and gemm.cuh.
+#include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -16,18 +18,26 @@ using namespace moe;
 
 namespace {
 
-// Two GEMM tile configurations, chosen per call from the tokens per expert:
-//   large: up to 160 token rows per tile (MMA N <= 160), 4-stage smem ring (54 KB stages);
-//   small: up to 32 token rows per tile, 5-stage ring (38 KB stages).  With a few tokens
-//   per expert the weight stream is the whole cost and the fifth stage keeps another
-//   16 KB weight tile per SM in flight.
-constexpr int kBN = 160, kStages = 4;
+// Routed grouped-GEMM tile configurations:
+//   WN (gemm.cuh): token rows on the MMA's M side, 256 weight rows on N, up to 128 token
+//   rows per tile, 4-stage smem ring (50 KB stages).  Each K block is one M=128 x N=256
+//   MMA whatever the token count, instead of two M=128 x N=n ones: the default while most
+//   experts have at most 128 rows (T*k <= 96*E), decode included;
+//   large: swap-AB (256 weight rows on M, up to 176 token rows on N), 4 stages (56 KB).
+//   Kimi-K3 prefill (T=8192) gives an expert ~146 +- 12 rows, so 176 keeps all but a
+//   handful of experts in one tile (with 160, one in eight was split in two half-full
+//   tiles, each costing as much tensor time as a full one);
+//   small: swap-AB with up to 32 token rows, 5 stages (38 KB): selectable, and the dense
+//   shared-expert GEMMs' tile for a few tokens per expert.
+constexpr int kBN = 176, kStages = 4;
+constexpr int kBNMid = 128, kStagesMid = 4;
 constexpr int kBNSmall = 32, kStagesSmall = 5;
 constexpr int kBNMin = kBNSmall;   // workspace sizing: the most tiles either configuration forms
 constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
 constexpr int kRouterStages = 3;
 constexpr int kRouterMaxCtas = 256;   // bound on split router tiles (sizes the partials)
+constexpr int kMaxDynSmem = 232448;   // opt-in dynamic shared memory per block (227 KB)
 constexpr int kSplitMaxCtas = 256;    // bound on split-K dense GEMM tiles (sizes their partials)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -63,11 +73,12 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Token-row maps for the grouped GEMM: box heights 32, 64, ... rows (one per tile size).
+// Token-row maps for the grouped GEMM: box heights 16, 32, ... rows (one per MMA N).
 bool make_bmaps(BMaps* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
                 uint64_t row_bytes, uint32_t box_inner) {
   for (int i = 0; i < MAX_BOX; ++i)
-    if (!make_map(&m->box[i], dt, base, inner, rows, row_bytes, box_inner, 32u * (i + 1))) return false;
+    if (!make_map(&m->box[i], dt, base, inner, rows, row_bytes, box_inner, (uint32_t)(BOX_ROWS * (i + 1))))
+      return false;
   return true;
 }
 
@@ -124,22 +135,26 @@ struct moe_plan_s {
   int bias_mode = MOE_BIAS_LOGIT;
   int flags = 0;
   const void* planes_of = nullptr;   // W_r the router planes were last split from
-  int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32 or 160
+  int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32, 128 or 176
   int last_bn = 0;            // token rows per tile in the last moe_forward
   int last_ksplit = 0;        // router K splits in the last moe_route
   int last_shared_split = 0;     // shared-expert gate/up K splits in the last moe_forward
   int last_shared_split_dn = 0;  // shared-expert down K splits in the last moe_forward
   size_t zpart_floats = 0;    // capacity of the router partials
-  // token rows per GEMM tile for a call with T tokens
+  // token rows per routed GEMM tile for a call with T tokens
   int tile_rows(int T) const {
     if (tile_n_opt) return tile_n_opt;
-    return (long long)T * k <= 8ll * E ? kBNSmall : kBN;   // <= 8 tokens per expert on average
+    const long long A = (long long)T * k;
+    return A <= 96ll * E ? kBNMid : kBN;  // WN while most experts fit 128 rows
   }
+  // token rows per tile of the dense (shared-expert, latent projection) GEMMs
+  int dense_rows(int T) const { return (long long)T * k <= 8ll * E ? kBNSmall : kBN; }
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
   size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
-      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_spart, o_xl, o_xn, o_yl, o_yr, total;
+      o_planes, o_rcnt, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_spart, o_theta, o_qbuf, o_xl, o_xn, o_yl,
+      o_yr, total;
   int dl = 0;              // latent option: expert width (0 = off)
   float eps_lat = 1e-5f;
   int tokens_per_chunk() const { return kPermThreads; }
@@ -165,6 +180,11 @@ static void carve(moe_plan_s* p) {
   p->zpart_floats = std::max((size_t)kRouterMaxCtas * kRouterBN * 128, (size_t)3 * p->T_max * p->E);
   p->o_zpart = take(p->zpart_floats * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
+  // fused router selection counters: [token tiles][expert tiles] splits done + [token tiles]
+  {
+    const size_t n_tt = (size_t)(std::max(p->T_max, 1) + kRouterBN - 1) / kRouterBN;
+    p->o_rcnt = take((n_tt * ((p->E + 127) / 128) + n_tt) * sizeof(int));
+  }
   p->o_xq = take(A * p->d);
   // token-side scale blocks, tile-major: at most A / bn + E group-tiles
   const size_t max_tiles = A / kBNMin + p->E + 1;
@@ -178,6 +198,10 @@ static void carve(moe_plan_s* p) {
   // split-K partials of the dense shared-expert GEMMs: ksplit * tiles <= kSplitMaxCtas, so
   // ksplit * T * M <= kSplitMaxCtas * kBN * 256 floats
   p->o_spart = take((size_t)kSplitMaxCtas * kBN * 256 * 4);
+  // Quantile Balancing inputs: each token's k-th largest key, and the quantiles handed to
+  // a bias rule
+  p->o_theta = take((size_t)std::max(p->T_max, 1) * 4);
+  p->o_qbuf = take((size_t)kMaxQuantLevels * p->E * 4);
   if (p->dl > 0) {   // latent option: x_l fp32, x_n bf16, y_l bf16 [T][dl], y_r fp32 [T][d]
     p->o_xl = take((size_t)p->T_max * p->dl * 4);
     p->o_xn = take((size_t)p->T_max * p->dl * 2);
@@ -202,11 +226,11 @@ static cudaError_t ensure_smem_attr(K kern, int bytes, std::atomic<uint64_t>& do
   return e;
 }
 
-template <int KIND, int EPI, int BN, int STAGES>
+template <int KIND, int EPI, int BN, int STAGES, bool WN = false>
 static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
                                    cudaStream_t s) {
-  using Cfg = GemmCfg<KIND, BN, STAGES>;
-  auto kern = gemm_kernel<KIND, EPI, BN, STAGES>;
+  using Cfg = GemmCfg<KIND, BN, STAGES, WN>;
+  auto kern = gemm_kernel<KIND, EPI, BN, STAGES, WN>;
   static std::atomic<uint64_t> attr_done{0};
   const cudaError_t e = ensure_smem_attr(kern, Cfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
@@ -215,9 +239,14 @@ static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, con
   return cudaGetLastError();
 }
 
+// Routed (block-scaled) GEMMs: the three configurations above.  Dense (bf16) GEMMs:
+// swap-AB with 32 or 176 token rows (128 is only ever asked for the routed ones).
 template <int KIND, int EPI>
 static cudaError_t launch_gemm(int bn, const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
                                cudaStream_t s) {
+  if constexpr (KIND == KIND_MX) {
+    if (bn == kBNMid) return launch_gemm_cfg<KIND, EPI, kBNMid, kStagesMid, true>(a, tA, tB, grid, s);
+  }
   if (bn == kBNSmall) return launch_gemm_cfg<KIND, EPI, kBNSmall, kStagesSmall>(a, tA, tB, grid, s);
   return launch_gemm_cfg<KIND, EPI, kBN, kStages>(a, tA, tB, grid, s);
 }
@@ -248,10 +277,8 @@ static GemmArgs base_args(const moe_plan_s* p) {
 }
 
 static cudaError_t set_smem_attrs() {
-  static std::atomic<uint64_t> place_done{0}, topk_done{0};
-  cudaError_t e = ensure_smem_attr(perm_place_kernel, 160 * 1024, place_done);
-  if (e == cudaSuccess) e = ensure_smem_attr(topk_sigmoid_kernel, 160 * 1024, topk_done);
-  return e;
+  static std::atomic<uint64_t> place_done{0};
+  return ensure_smem_attr(perm_place_kernel, 160 * 1024, place_done);
 }
 
 // histogram -> scan -> placement into the plan workspace
@@ -415,9 +442,16 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   // MOE_BIAS_SELECT_ONLY: z stays unbiased; the bias only enters the top-k key
   const bool select_only = p->bias_mode == MOE_BIAS_SELECT_ONLY;
   ra.bias = select_only ? nullptr : bias;
+  ra.sel_bias = select_only ? bias : nullptr;
   ra.z = z;
   ra.zpart = p->at<float>(p->o_zpart);
   ra.status = p->at<unsigned int>(p->o_status);
+  ra.k = p->k;
+  ra.idx = idx;
+  ra.w = w;
+  const int n_tt = (T + kRouterBN - 1) / kRouterBN;
+  ra.cnt_split = p->at<int>(p->o_rcnt);
+  ra.cnt_tile = ra.cnt_split + (size_t)n_tt * ra.m_tiles;
   {
     // Split K (i) when the expert x token tiles would fill less than half the SMs, so that
     // the plane reads (3 x E x d bf16) spread over the whole GPU, and (ii) otherwise by up
@@ -446,25 +480,21 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
+    // the fused selection keeps one E-float row per epilogue warp after the pipeline
+    ra.topk_warps = std::min(8, (kMaxDynSmem - RC::SMEM_BYTES) / (E * 4));
+    if (ra.topk_warps < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+    const int smem = RC::SMEM_BYTES + ra.topk_warps * E * 4;
     static std::atomic<uint64_t> router_done{0};
-    if (ensure_smem_attr(kern, RC::SMEM_BYTES, router_done) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ensure_smem_attr(kern, kMaxDynSmem, router_done) != cudaSuccess) return MOE_ERR_CUDA;
     const int tiles = base_tiles * ra.ksplit;
     p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
-    kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
-    if (ra.ksplit > 1) {
-      const long long n = (long long)T * E;
-      router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ra.zpart, ra.ksplit, ra.bias, T, E, z);
-    }
+    // the selection counters start from zero every call
+    if (cudaMemsetAsync(ra.cnt_split, 0, ((size_t)n_tt * ra.m_tiles + n_tt) * sizeof(int), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    kern<<<std::min(tiles, p->num_sms), 320, smem, s>>>(ra, tA, tB);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
-  if (set_smem_attrs() != cudaSuccess) return MOE_ERR_CUDA;
-  const int wpb = 8;
-  p->prof.begin(MOE_STAGE_TOPK, s);
-  topk_sigmoid_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * E * 4, s>>>(
-      z, select_only ? bias : nullptr, T, E, p->k, idx, w);
-  p->prof.end(s);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   p->last_T = T;
   return MOE_OK;
 }
@@ -515,7 +545,8 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
   const int d = p->d, E = p->E, k = p->k, I = p->I, Is = p->Is;
   const int de = lat ? p->dl : d;   // width the routed experts act on
   const int A = T * k;
-  const int bn = p->tile_rows(T);
+  const int bn = p->tile_rows(T);                    // routed GEMM tiles
+  const int dbn = p->dense_rows(T);                  // dense GEMM tiles
 
   // latent option: x_l = x W_ld^T, x_n = bf16(RMSNorm(x_l) * gamma) feeds the experts
   const void* xin = x;
@@ -523,7 +554,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     float* xl = p->at<float>(p->o_xl);
     __nv_bfloat16* xn = p->at<__nv_bfloat16>(p->o_xn);
     p->prof.begin(MOE_STAGE_LATENT_IN, s);
-    if (dense_bf16_f32(p, lat->w_down, de, x, d, T, xl, bn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dense_bf16_f32(p, lat->w_down, de, x, d, T, xl, dbn, s) != cudaSuccess) return MOE_ERR_CUDA;
     rmsnorm_bf16_kernel<<<T, 256, 0, s>>>(xl, lat->gamma, de, p->eps_lat, xn);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -630,7 +661,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     a.B_rows = T;
     a.out0 = hsh;
     a.ld_out = Is;
-    int tiles = ((T + bn - 1) / bn) * a.m_tiles;
+    int tiles = ((T + dbn - 1) / dbn) * a.m_tiles;
     float* spart = p->at<float>(p->o_spart);
     p->prof.begin(MOE_STAGE_SHARED_GATE_UP, s);
     const int ks_gu = dense_ksplit(p, tiles, a.k_tiles, (size_t)T * 2 * Is);
@@ -641,7 +672,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
       a.split_stride = (long long)T * 2 * Is;
       a.out0 = spart;
       a.ld_out = 2 * Is;
-      if (launch_gemm<KIND_BF16, EPI_F32>(bn, a, tA, tB, std::min(tiles * ks_gu, p->num_sms), s) != cudaSuccess)
+      if (launch_gemm<KIND_BF16, EPI_F32>(dbn, a, tA, tB, std::min(tiles * ks_gu, p->num_sms), s) != cudaSuccess)
         return MOE_ERR_CUDA;
       const long long n = (long long)T * Is;
       if (p->act == MOE_ACT_CLAMPED_SWIGLU)
@@ -651,8 +682,8 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
       if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
-          ? launch_gemm<KIND_BF16, EPI_GLU_BF16_CLAMPED>(bn, a, tA, tB, std::min(tiles, p->num_sms), s)
-          : launch_gemm<KIND_BF16, EPI_GLU_BF16>(bn, a, tA, tB, std::min(tiles, p->num_sms), s);
+          ? launch_gemm<KIND_BF16, EPI_GLU_BF16_CLAMPED>(dbn, a, tA, tB, std::min(tiles, p->num_sms), s)
+          : launch_gemm<KIND_BF16, EPI_GLU_BF16>(dbn, a, tA, tB, std::min(tiles, p->num_sms), s);
       if (e != cudaSuccess)
         return MOE_ERR_CUDA;
     }
@@ -673,7 +704,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     b.B_rows = T;
     b.out0 = ys;
     b.ld_out = d;
-    tiles = ((T + bn - 1) / bn) * b.m_tiles;
+    tiles = ((T + dbn - 1) / dbn) * b.m_tiles;
     p->prof.begin(MOE_STAGE_SHARED_DOWN, s);
     const int ks_dn = dense_ksplit(p, tiles, b.k_tiles, (size_t)T * d);
     if (ks_dn > 1) {
@@ -681,13 +712,13 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
       b.k_per = (b.k_tiles + ks_dn - 1) / ks_dn;
       b.split_stride = (long long)T * d;
       b.out0 = spart;
-      if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles * ks_dn, p->num_sms), s) != cudaSuccess)
+      if (launch_gemm<KIND_BF16, EPI_F32>(dbn, b, tA2, tB2, std::min(tiles * ks_dn, p->num_sms), s) != cudaSuccess)
         return MOE_ERR_CUDA;
       const long long n = (long long)T * d;
       split_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_dn, n, b.split_stride, ys);
       if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     } else {
-      if (launch_gemm<KIND_BF16, EPI_F32>(bn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
+      if (launch_gemm<KIND_BF16, EPI_F32>(dbn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
     p->last_shared_split_dn = ks_dn;
@@ -711,7 +742,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
         O, nullptr, w, p->at<int>(p->o_inv), T, de, k, yl);
     p->prof.end(s);
     p->prof.begin(MOE_STAGE_LATENT_OUT, s);
-    if (dense_bf16_f32(p, lat->w_up, d, yl, de, T, yr, bn, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dense_bf16_f32(p, lat->w_up, d, yl, de, T, yr, dbn, s) != cudaSuccess) return MOE_ERR_CUDA;
     const long long n = (long long)T * d;
     add_bf16_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, s>>>(yr, ys, n, (__nv_bfloat16*)y);
     p->prof.end(s);
@@ -796,6 +827,51 @@ moe_status_t moe_pack_shared_bf16(int d, int Is, const void* wg, const void* wu,
   return MOE_OK;
 }
 
+moe_status_t moe_route_margin_quantiles(moe_plan_t p, const float* logits, const float* select_bias, int T,
+                                        const double* levels, int n_levels, float* quantiles, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  if (T <= 0 || n_levels <= 0 || !logits || !levels || !quantiles) return MOE_ERR_INVALID_ARG;
+  if (T > p->T_max || n_levels > kMaxQuantLevels) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(logits, 4) || !aligned(quantiles, 4) || (select_bias && !aligned(select_bias, 4)))
+    return MOE_ERR_ALIGNMENT;
+  QuantRanks rk;
+  memset(&rk, 0, sizeof(rk));
+  for (int i = 0; i < n_levels; ++i) {
+    const double q = levels[i];
+    if (!(q >= 0.0 && q <= 1.0)) return MOE_ERR_INVALID_ARG;   // also rejects NaN
+    const double j = std::ceil(q * (double)T);
+    rk.r[i] = (int)std::min<double>(std::max<double>(j, 1.0), (double)T);
+  }
+  cudaStream_t s = S(stream);
+  static std::atomic<uint64_t> kth_done{0};
+  if (ensure_smem_attr(kth_key_kernel, 160 * 1024, kth_done) != cudaSuccess) return MOE_ERR_CUDA;
+  float* theta = p->at<float>(p->o_theta);
+  const int wpb = 8;
+  kth_key_kernel<<<(T + wpb - 1) / wpb, wpb * 32, (size_t)wpb * p->E * 4, s>>>(logits, select_bias, T, p->E, p->k,
+                                                                               theta);
+  margin_quantile_kernel<<<dim3((p->E + 31) / 32, n_levels), kQuantThreads, 0, s>>>(logits, select_bias, theta, T,
+                                                                                     p->E, rk, quantiles);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_quantile_balance(moe_plan_t p, const float* logits, const float* bias, int T,
+                                  const double* levels, int n_levels, moe_bias_rule_t rule, void* user,
+                                  float* bias_next, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!p->ws) return MOE_ERR_NOT_INITIALIZED;
+  if (!rule || !bias || !bias_next) return MOE_ERR_INVALID_ARG;
+  if (!aligned(bias, 4) || !aligned(bias_next, 4)) return MOE_ERR_ALIGNMENT;
+  // the margins read the selection key: z + b in the select-only mode, z otherwise (a
+  // logit bias is already inside z)
+  const float* sel = p->bias_mode == MOE_BIAS_SELECT_ONLY ? bias : nullptr;
+  float* q = p->at<float>(p->o_qbuf);
+  const moe_status_t st = moe_route_margin_quantiles(p, logits, sel, T, levels, n_levels, q, stream);
+  if (st != MOE_OK) return st;
+  rule(q, n_levels, p->E, bias, bias_next, stream, user);
+  return MOE_OK;
+}
+
 moe_status_t moe_plan_set_option(moe_plan_t p, int option, int value) {
   if (!p) return MOE_ERR_INVALID_ARG;
   switch (option) {
@@ -807,7 +883,7 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int option, int value) {
       p->pf_b = value != 0;
       return MOE_OK;
     case MOE_OPT_TILE_N:
-      if (value != 0 && value != kBNSmall && value != kBN) return MOE_ERR_INVALID_ARG;
+      if (value != 0 && value != kBNSmall && value != kBNMid && value != kBN) return MOE_ERR_INVALID_ARG;
       p->tile_n_opt = value;
       return MOE_OK;
   }
@@ -873,6 +949,7 @@ moe_status_t moe_debug_buffer(moe_plan_t p, int which, void** ptr, size_t* bytes
     case 4: off = p->o_O; n = A * p->d * 2; break;
     case 5: off = p->o_ys; n = T * p->d * 4; break;
     case 6: off = p->o_logits; n = T * p->E * 4; break;
+    case 7: off = p->o_qbuf; n = (size_t)kMaxQuantLevels * p->E * 4; break;
     default: return MOE_ERR_INVALID_ARG;
   }
   *ptr = p->ws + off;

@@ -26,6 +26,17 @@
 // warp 11 copies each stage's scale factors into TMEM (KIND_MX), warp 1 owns TMEM and one
 // lane issues the MMAs, two K tiles per round, warps 2..9 run the epilogue (lane quarter =
 // warp % 4).  The producers and the scale warp complete the same stage independently.
+//
+// Orientation WN (KIND_MX, a few tokens per expert): the token rows are the MMA's M side
+// (128 lanes, of which the tile's rows are the first n) and all 256 weight rows of the tile
+// are its N side, so each K block is one M=128 x N=256 instruction instead of two M=128 x
+// N=n ones.  Issued back to back from one thread, a block-scaled M=128 tcgen05.mma takes
+// the same time for every N from 16 to 256 (measured: ~135 cycles at 1965 MHz, about the
+// N=256 execution time), so with few tokens this halves the time per weight byte, and the
+// weight stream is what the kernel is there for.
+// The accumulator is then tokens x (gate | up) or tokens x output channels; the epilogue
+// reads a token row per thread.  Shared memory, producers and scale copies are as above
+// (the weight scales become the B side's, the token scales the A side's).
 #pragma once
 #include "ptx.cuh"
 #include "tiling.cuh"
@@ -76,7 +87,7 @@ struct GemmArgs {
   long long split_stride;
 };
 
-template <int KIND, int BN_MAX, int STAGES>
+template <int KIND, int BN_MAX, int STAGES, bool WN = false>
 struct GemmCfg {
   static constexpr int BM = 256;                               // two 128-row halves
   static constexpr int BK = KIND == KIND_MX ? 128 : 64;        // elements per K tile (128 B rows)
@@ -89,15 +100,20 @@ struct GemmCfg {
   static constexpr int A_TX = KIND == KIND_MX ? BM * BK / 2 : BM * BK * 2;  // global bytes
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
   // scale factors in TMEM, one 16-column buffer per pipeline stage:
-  //   A: 4 columns per 128-row half (+0, +4), B: 4 columns per 128 token rows (+8, +12)
-  static constexpr int TMEM_SF = 2 * BN_MAX;
+  //   weights: 4 columns per 128-row half (+0, +4), tokens: 4 columns per 128 rows (+8, +12)
+  // after the accumulator (two halves of BN_MAX columns, or WN: 256 columns)
+  static constexpr int TMEM_SF = WN ? 256 : 2 * BN_MAX;
   static constexpr int TMEM_COLS = 512;
   static constexpr int NUM_THREADS = 384;
-  static_assert(BN_MAX % 32 == 0 && BN_MAX <= 256, "BN_MAX");
+  static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "BN_MAX");
   static_assert(SFB_ATOMS <= 2, "scale buffer holds two B atoms");
   static_assert(TMEM_SF + 16 * STAGES <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // WN: the M=128 MMA reads 128 token rows (16 KB) from the token region whatever the
+  // tile's row count, so the region must hold 128 rows (rows past the tile's are stale and
+  // only reach accumulator lanes that nothing reads)
+  static_assert(!WN || (KIND == KIND_MX && BN_MAX == 128), "WN: block-scaled, a 128-row token region");
 };
 
 struct TileInfo {
@@ -208,17 +224,18 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Token-row tensor maps with box heights 32, 64, ..., 32 * MAX_BOX rows.
-constexpr int MAX_BOX = 8;
+// Token-row tensor maps with box heights 16, 32, ..., 16 * MAX_BOX rows (one per MMA N).
+constexpr int BOX_ROWS = 16;
+constexpr int MAX_BOX = 16;
 struct BMaps {
   CUtensorMap box[MAX_BOX];
 };
 
-template <int KIND, int EPI, int BN_MAX, int STAGES>
+template <int KIND, int EPI, int BN_MAX, int STAGES, bool WN = false>
 __global__ void __launch_bounds__(384, 1)
     gemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA,
                 const __grid_constant__ BMaps tmB) {
-  using C = GemmCfg<KIND, BN_MAX, STAGES>;
+  using C = GemmCfg<KIND, BN_MAX, STAGES, WN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ctrl = smem + STAGES * C::STAGE_BYTES;
@@ -234,6 +251,10 @@ __global__ void __launch_bounds__(384, 1)
   // Fill counters for the abort cleanup: [0] weight producer, [1] token producer, [2] scale
   // warp (sf_full fills consumed = full-barrier arrivals made), [3] MMA (fills consumed).
   int* fills = (int*)(tmem_holder + 2);
+  // MMA N of the tile a stage belongs to, written by the token producer before it arrives
+  // on the stage's full barrier (so the MMA thread never decodes routed tiles itself: that
+  // takes dependent global loads, a binary search over the expert tile table)
+  int* stage_n = fills + 4;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -333,7 +354,7 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) fills[0] = nfill;
   } else if (warp == 10) {
     // ------------------------------------------------------------- producer: token rows
-    // One TMA box of the tile's rows (box height 32 * nB, nB = ceil(n_mma / 32)) and
+    // One TMA box of the tile's n_mma rows (a multiple of 16: box height 16 * nB) and
     // (KIND_MX) one bulk copy of the tile's scale atoms for this K tile.
     const uint64_t pol_b = policy_evict_last();   // token rows are shared by the m-tiles
     int stage = 0;
@@ -343,7 +364,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
-      const int nB = (ti.n_mma + 31) >> 5;
+      const int nB = ti.n_mma / BOX_ROWS;
       for (int kt = ti.kb; kt < ti.ke; ++kt) {
         if (lane == 0) ok = mbar_wait(smem_u32(empty_bar + stage), phase ^ 1, args.status, abort_flag);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -351,7 +372,8 @@ __global__ void __launch_bounds__(384, 1)
         uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
         const uint32_t fb = smem_u32(full_bar + stage);
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, nB * 4096);
+          stage_n[stage] = ti.n_mma;
+          mbar_arrive_expect_tx(fb, nB * BOX_ROWS * 128);
           tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
           if constexpr (KIND == KIND_MX) {
             const int sfb_bytes = ((ti.n_mma + 127) >> 7) * 512;
@@ -399,7 +421,7 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t sfb_desc = sfa_desc + (uint64_t)(C::SFA_BYTES >> 4);
           const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
           tc_cp_32x128b_warpx4(tsf, sfa_desc);
-          if (h1) tc_cp_32x128b_warpx4(tsf + 4, sfa_desc + (uint64_t)(512 >> 4));
+          if (h1 || WN) tc_cp_32x128b_warpx4(tsf + 4, sfa_desc + (uint64_t)(512 >> 4));
           tc_cp_32x128b_warpx4(tsf + 8, sfb_desc);
           if (atoms > 1) tc_cp_32x128b_warpx4(tsf + 12, sfb_desc + (uint64_t)(512 >> 4));
           tc_commit(smem_u32(full_bar + stage));
@@ -422,37 +444,45 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       int nfill = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        // The tile's K range and weight m-tile are arithmetic; its MMA N comes with its
+        // first stage (stage_n, below).
         TileInfo ti;
-        gemm_decode_tile(args, BN_MAX, t, ti);
+        if (args.dense_rows >= 0) {
+          gemm_decode_tile(args, BN_MAX, t, ti);
+        } else {
+          ti.mt = t % args.m_tiles;
+          ti.kb = 0;
+          ti.ke = args.k_tiles;
+        }
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
-        // Everything the MMAs of a stage need except the stage offset is fixed per tile:
-        // the issue loop below only adds constants (the tcgen05.mma issue rate is set by
-        // how fast this one thread can form its operands).
         uint32_t idesc[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          idesc[j] = KIND == KIND_MX ? idesc_mx_e2m1_e4m3(128, ti.n_mma, j, j) : idesc_bf16(128, ti.n_mma);
-        ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // the 8 MMAs (4 K-blocks x 2 halves) of the K tile held by smem stage st
+        bool first = true;
+        // the MMAs of the K tile held by smem stage st: 4 K-blocks x 2 halves (WN: 4 K-blocks)
         auto issue_stage = [&](int st, uint32_t acc0) {
           const uint64_t a_desc = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
           const uint64_t b_desc = a_desc + (uint64_t)(C::A_BYTES >> 4);
           const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * st;
+          if constexpr (WN) {
+            // token tile (A, M=128) x all 256 weight rows (B, N=256), one MMA per K block
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 4; ++j)
+              mma_mxf8f6f4(tmem_base, b_desc + (uint64_t)((32 * j) >> 4), a_desc + (uint64_t)((32 * j) >> 4), idesc[j],
+                           (tsf + 8) | ((uint32_t)j << 30), tsf | ((uint32_t)j << 30), j > 0 ? 1u : acc0);
+          } else {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (h == 1 && !h1) continue;
-              const uint64_t adesc = a_desc + (uint64_t)((h * 16384 + 32 * j) >> 4);
-              const uint64_t bdesc = b_desc + (uint64_t)((32 * j) >> 4);
-              const uint32_t acc = j > 0 ? 1u : acc0;
-              if constexpr (KIND == KIND_MX)
-                mma_mxf8f6f4(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], (tsf + 4 * h) | ((uint32_t)j << 30),
-                             (tsf + 8) | ((uint32_t)j << 30), acc);
-              else
-                mma_bf16(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], acc);
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !h1) continue;
+                const uint64_t adesc = a_desc + (uint64_t)((h * 16384 + 32 * j) >> 4);
+                const uint64_t bdesc = b_desc + (uint64_t)((32 * j) >> 4);
+                const uint32_t acc = j > 0 ? 1u : acc0;
+                if constexpr (KIND == KIND_MX)
+                  mma_mxf8f6f4(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], (tsf + 4 * h) | ((uint32_t)j << 30),
+                               (tsf + 8) | ((uint32_t)j << 30), acc);
+                else
+                  mma_bf16(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], acc);
+              }
             }
           }
         };
@@ -471,6 +501,20 @@ __global__ void __launch_bounds__(384, 1)
             if (ok) ++nfill;
           }
           if (!ok) break;
+          if (first) {
+            // Everything the MMAs of a stage need except the stage offset is fixed per
+            // tile: the issue loop only adds constants (the tcgen05.mma issue rate is set
+            // by how fast this one thread can form its operands).
+            const int n_mma = stage_n[stage];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              idesc[j] = WN ? idesc_mx_e4m3_e2m1(128, 256, j, j)
+                            : (KIND == KIND_MX ? idesc_mx_e2m1_e4m3(128, n_mma, j, j) : idesc_bf16(128, n_mma));
+            // the accumulator is free once the epilogue has drained the previous tile
+            ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
+            if (!ok) break;
+            first = false;
+          }
           tc_fence_after();
           issue_stage(stage, kt > ti.kb ? 1u : 0u);
           tc_commit(smem_u32(empty_bar + stage));
@@ -515,12 +559,104 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(acc_empty));
       };
-      if constexpr (EpiTraits<EPI>::glu) {
+      if constexpr (WN) {
+        // TMEM lane = token row of the tile (quarter q: rows 32q..32q+31), column = weight
+        // row of the tile.  tcgen05.ld is warp-wide, so a warp without valid rows only
+        // releases TMEM.
+        const int r = q * 32 + lane;
+        const bool any = q * 32 < ti.n_valid;
+        const bool row_ok = r < ti.n_valid;
+        const size_t row = (size_t)(ti.row0 + r);
+        if constexpr (EpiTraits<EPI>::glu) {
+          // columns c < 128: gate of channel mt*128 + c; 128 + c: its up.  Warp half `sub`
+          // takes the 32-channel blocks 2 sub and 2 sub + 1.
+          float a[2][32];
+          if (any) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int b = 2 * sub + i;
+              uint32_t g0[16], g1[16], u0[16], u1[16];
+              tmem_ld16(lane_base + 32 * b, g0);
+              tmem_ld16(lane_base + 32 * b + 16, g1);
+              tmem_ld16(lane_base + 128 + 32 * b, u0);
+              tmem_ld16(lane_base + 128 + 32 * b + 16, u1);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                a[i][j] = glu_f<EpiTraits<EPI>::act>(__uint_as_float(g0[j]), __uint_as_float(u0[j]));
+                a[i][16 + j] = glu_f<EpiTraits<EPI>::act>(__uint_as_float(g1[j]), __uint_as_float(u1[j]));
+              }
+            }
+          }
+          release_tmem();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int b = 2 * sub + i;
+              const size_t col = (size_t)ti.mt * 128 + 32 * b;
+              if constexpr (EpiTraits<EPI>::mx8_out) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(a[i][j]));
+                const int e = mx_exp_e4m3(__float_as_uint(amax));
+                const float sc = __uint_as_float((uint32_t)(127 - e) << 23);
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  w[j] = f32x2_to_e4m3x2(a[i][4 * j] * sc, a[i][4 * j + 1] * sc) |
+                         (f32x2_to_e4m3x2(a[i][4 * j + 2] * sc, a[i][4 * j + 3] * sc) << 16);
+                uint4* dst = (uint4*)((uint8_t*)args.out0 + row * args.ld_out + col);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                // scale byte for the down GEMM: K tile mt, block b, tile-major
+                ((uint8_t*)args.out1)[((size_t)ti.gt * args.m_tiles + ti.mt) * SF_TILE_BYTES + sf_atom_offset(r) + b] =
+                    (uint8_t)(e + 127);
+              } else {
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const __nv_bfloat162 p2 = __floats2bfloat162_rn(a[i][2 * j], a[i][2 * j + 1]);
+                  w[j] = *(const uint32_t*)&p2;
+                }
+                uint4* dst = (uint4*)((__nv_bfloat16*)args.out0 + row * args.ld_out + col);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+              }
+            }
+          }
+        } else {
+          // output channels mt*256 + 128 sub + c, c < 128, rounded to bf16 (EPI_BF16)
+          static_assert(EPI == EPI_BF16, "WN epilogues: GLU (MXFP8 / bf16) or bf16");
+          const int ch0 = ti.mt * 256 + 128 * sub;
+          const bool half_ok = ch0 < args.M_total;
+          uint32_t v[64];
+          if (any && half_ok) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t rr[16];
+              tmem_ld16(lane_base + 128 * sub + 16 * c, rr);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * j]), __uint_as_float(rr[2 * j + 1]));
+                v[8 * c + j] = *(const uint32_t*)&p2;
+              }
+            }
+          }
+          release_tmem();
+          if (half_ok && row_ok) {
+            uint4* dst = (uint4*)((uint16_t*)args.out0 + row * args.ld_out + ch0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+      } else if constexpr (EpiTraits<EPI>::glu) {
         // a = glu(g, u) for this warp's chunks (c = sub + 2 i) straight out of TMEM;
         // TMEM goes back to the MMA warp before the quantisation and stores.
-        float a[CH / 2][16];
+        constexpr int CH2 = (CH + 1) / 2;   // this warp's chunks: c = sub + 2 i
+        float a[CH2][16];
 #pragma unroll
-        for (int i = 0; i < CH / 2; ++i) {
+        for (int i = 0; i < CH2; ++i) {
           const int c = sub + 2 * i;
           if (c < nchunks) {
             uint32_t g[16], u[16];
@@ -534,7 +670,7 @@ __global__ void __launch_bounds__(384, 1)
         release_tmem();
         const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
 #pragma unroll
-        for (int i = 0; i < CH / 2; ++i) {
+        for (int i = 0; i < CH2; ++i) {
           const int c = sub + 2 * i;
           if (c >= nchunks) break;
 #pragma unroll

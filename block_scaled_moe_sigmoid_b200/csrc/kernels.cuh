@@ -306,42 +306,16 @@ __global__ void perm_place_kernel(const int* __restrict__ idx, int T, int k, int
 }
 
 // ---------------------------------------------------------------- top-k
-// K-split router logits: z[t][e] = (sum over s, in order, of zpart[s][t][e]) + bias[e].
-// One thread per logit; the partials are fetched eight at a time so that the loads
-// overlap, and added in split order.
-__global__ void router_reduce_kernel(const float* __restrict__ zpart, int nsplit,
-                                     const float* __restrict__ bias, int T, int E, float* __restrict__ z) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long n = (long long)T * E;
-  if (i >= n) return;
-  float v = 0.0f;
-  for (int s0 = 0; s0 < nsplit; s0 += 8) {
-    float p[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) p[q] = s0 + q < nsplit ? __ldg(zpart + (size_t)(s0 + q) * n + i) : 0.0f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (s0 + q < nsplit) v = (s0 + q == 0) ? p[q] : v + p[q];
-  }
-  if (bias) v += __ldg(bias + (int)(i % E));
-  z[i] = v;
-}
-
-// One warp per token: k rounds of a warp arg-max over the logits (descending value,
-// lower index on ties), then sigmoid weights renormalised to sum 1.
-// select_bias != NULL (select-only bias): the arg-max runs on the key z + b (fp32), the
-// weights still come from sigmoid(z).
-__global__ void topk_sigmoid_kernel(const float* __restrict__ z, const float* __restrict__ select_bias,
-                                    int T, int E, int k, int* __restrict__ idx_out,
-                                    float* __restrict__ w_out) {
-  extern __shared__ float zs[];  // [warps][E]
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + w;
-  if (t >= T) return;
-  float* row = zs + (size_t)w * E;
-  // row holds the selection key (z, or z + b in select-only mode)
+// Selection for one token, by one warp: key = z (+ select_bias in the select-only mode,
+// fp32); k rounds of a warp arg-max over the keys (descending value, lower index on equal
+// values), then w_j = s_j / sum of the selected s, s = sigmoid(z).  row: the warp's
+// shared-memory scratch of E floats.  z is read through L2 (__ldcg): it may have been
+// written by other CTAs of the same kernel.
+__device__ __forceinline__ void topk_sigmoid_row(const float* __restrict__ z_row, const float* __restrict__ select_bias,
+                                                 int E, int k, float* row, int* __restrict__ idx_out,
+                                                 float* __restrict__ w_out, int lane) {
   for (int e = lane; e < E; e += 32)
-    row[e] = select_bias ? __ldg(z + (size_t)t * E + e) + __ldg(select_bias + e) : __ldg(z + (size_t)t * E + e);
+    row[e] = select_bias ? __ldcg(z_row + e) + __ldg(select_bias + e) : __ldcg(z_row + e);
   __syncwarp();
   float ssum = 0.0f, my_s = 0.0f;
   int my_i = -1;
@@ -358,7 +332,7 @@ __global__ void topk_sigmoid_kernel(const float* __restrict__ z, const float* __
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    const float zsel = select_bias ? __ldg(z + (size_t)t * E + bi) : bv;
+    const float zsel = select_bias ? __ldcg(z_row + bi) : bv;
     const float s = 1.0f / (1.0f + expf(-zsel));
     ssum += s;
     if (lane == r) { my_s = s; my_i = bi; }
@@ -366,9 +340,10 @@ __global__ void topk_sigmoid_kernel(const float* __restrict__ z, const float* __
     __syncwarp();
   }
   if (lane < k) {
-    idx_out[(size_t)t * k + lane] = my_i;
-    w_out[(size_t)t * k + lane] = my_s / ssum;
+    idx_out[lane] = my_i;
+    w_out[lane] = my_s / ssum;
   }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------- combine
@@ -560,6 +535,110 @@ __global__ void router_split_kernel(const float* __restrict__ W, int d, int E,
       row[2 * d + i] = lo;
     }
   }
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------- Quantile Balancing inputs
+// Routing margin m[t][e] = key[t][e] - theta[t], with key = z (+ b in the select-only
+// mode, formed in fp32) and theta[t] the token's k-th largest key; the per-expert quantile
+// at level q is the order statistic of rank j = clamp(ceil(q T), 1, T) of m[:, e].
+
+// One warp per token: theta[t] = the k-th largest key (k rounds of a warp arg-max, lower
+// index first on equal keys, as in the selection).
+__global__ void kth_key_kernel(const float* __restrict__ z, const float* __restrict__ select_bias, int T,
+                               int E, int k, float* __restrict__ theta) {
+  extern __shared__ float keys[];  // [warps][E]
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + w;
+  if (t >= T) return;
+  float* row = keys + (size_t)w * E;
+  for (int e = lane; e < E; e += 32)
+    row[e] = select_bias ? __ldg(z + (size_t)t * E + e) + __ldg(select_bias + e) : __ldg(z + (size_t)t * E + e);
+  __syncwarp();
+  float bv = -INFINITY;
+  for (int r = 0; r < k; ++r) {
+    bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      const float v = row[e];
+      if (v > bv) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) row[bi] = -INFINITY;
+    __syncwarp();
+  }
+  if (lane == 0) theta[t] = bv;
+}
+
+// fp32 -> uint32 with the same order (negatives flipped whole, positives' sign bit set).
+__device__ __forceinline__ uint32_t f32_order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float f32_from_order_key(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Exact order statistics of the margins by radix select, 8 bits a pass from the top.
+// CTA (group g, level l): experts 32 g .. 32 g + 31 (lane = expert within the group), rank
+// ranks[l].  256 threads; each warp walks tokens w, w + 8, ... and reads one 128-byte run
+// of a token's logits per step.
+constexpr int kQuantThreads = 256;
+constexpr int kMaxQuantLevels = 16;
+struct QuantRanks {
+  int r[kMaxQuantLevels];   // 1-based ranks, one per level
+};
+__global__ void __launch_bounds__(kQuantThreads)
+    margin_quantile_kernel(const float* __restrict__ z, const float* __restrict__ select_bias,
+                           const float* __restrict__ theta, int T, int E, const QuantRanks ranks,
+                           float* __restrict__ out) {
+  __shared__ uint32_t hist[32][257];
+  __shared__ uint32_t s_prefix[32], s_rank[32];
+  const int g = blockIdx.x, lvl = blockIdx.y;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = g * 32 + lane;
+  const bool e_ok = e < E;
+  const float b = (select_bias && e_ok) ? __ldg(select_bias + e) : 0.0f;
+  if (threadIdx.x < 32) {
+    s_prefix[threadIdx.x] = 0u;
+    s_rank[threadIdx.x] = (uint32_t)ranks.r[lvl];   // 1-based rank within the column
+  }
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = threadIdx.x; i < 32 * 257; i += blockDim.x) (&hist[0][0])[i] = 0u;
+    __syncthreads();
+    const uint32_t prefix = s_prefix[lane];
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (32 - 8 * pass));
+    if (e_ok) {
+      for (int t = w; t < T; t += blockDim.x >> 5) {
+        const float key = select_bias ? __ldg(z + (size_t)t * E + e) + b : __ldg(z + (size_t)t * E + e);
+        const uint32_t u = f32_order_key(key - __ldg(theta + t));
+        if ((u & hi_mask) == prefix) atomicAdd(&hist[lane][(u >> shift) & 255u], 1u);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32 && g * 32 + (int)threadIdx.x < E) {
+      uint32_t r = s_rank[threadIdx.x], digit = 0;
+      for (; digit < 255; ++digit) {
+        const uint32_t c = hist[threadIdx.x][digit];
+        if (r <= c) break;
+        r -= c;
+      }
+      s_rank[threadIdx.x] = r;
+      s_prefix[threadIdx.x] |= digit << shift;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < 32 && g * 32 + (int)threadIdx.x < E)
+    out[(size_t)lvl * E + g * 32 + threadIdx.x] = f32_from_order_key(s_prefix[threadIdx.x]);
 }
 
 }  // namespace moe

@@ -243,6 +243,18 @@ __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, uint32_t
          | ((sfa_id & 3u) << 29);      // A scale-factor id
 }
 
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A = E4M3, B = E2M1, E8M0 scales.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_e2m1(int M, int N, uint32_t sfa_id,
+                                                         uint32_t sfb_id) {
+  return ((sfb_id & 3u) << 4)          // B scale-factor id (byte within the TMEM word)
+         | (0u << 7)                   // A format E4M3
+         | (5u << 10)                  // B format E2M1
+         | ((uint32_t)(N >> 3) << 17)  // N / 8
+         | (1u << 23)                  // scale format E8M0
+         | ((uint32_t)(M >> 4) << 24)  // M / 16
+         | ((sfa_id & 3u) << 29);      // A scale-factor id
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }

@@ -11,10 +11,17 @@
 // Tile: 128 experts (MMA M = lanes) x up to RBN tokens (MMA N = columns) x a range of
 // 64-column chains.  With few tokens (decode) the expert x token tiles alone would occupy
 // a handful of SMs, so K is split: split s covers chains [s * chains_per, ...) and writes
-// its fp32 partial to zpart[s]; the top-k kernel adds the partials in split order and the
-// bias.  Roles as in gemm.cuh: warp 0 loads (TMA), warp 1 issues MMAs, warps 2..9 drain
-// and store.
+// its fp32 partial to zpart[s].  Roles as in gemm.cuh: warp 0 loads (TMA), warp 1 issues
+// MMAs, warps 2..9 drain and store.
+//
+// Selection is fused: the CTA that completes the last split of a (token tile, expert tile)
+// adds the partials in split order plus the bias and writes z; the CTA that completes the
+// last expert tile of a token tile has every logit of those tokens and runs the sigmoid
+// top-k (topk_sigmoid_row) for them.  "Last" is decided by counters (atomicAdd after a
+// fence of the CTA's stores); nothing waits on another CTA, and the counters are zeroed
+// before the launch.
 #pragma once
+#include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -24,10 +31,17 @@ struct RouterArgs {
   int m_tiles;     // ceil(E / 128)
   int ksplit;      // K splits (1: no split)
   int chains_per;  // 64-column chains per split
-  const float* bias;
-  float* z;        // [T][E] (ksplit == 1)
+  const float* bias;        // logit bias added to z, or NULL
+  const float* sel_bias;    // select-only bias (selection key z + b), or NULL
+  float* z;        // [T][E] logits
   float* zpart;    // [ksplit][T][E] partials without bias (ksplit > 1)
   unsigned int* status;
+  int k;           // experts per token
+  int* idx;        // [T][k] selected experts, descending key
+  float* w;        // [T][k] renormalised sigmoid weights
+  int* cnt_split;  // [token tiles][m_tiles] splits done (zeroed before the launch)
+  int* cnt_tile;   // [token tiles] expert tiles done (zeroed before the launch)
+  int topk_warps;  // epilogue warps with an E-float selection row in shared memory
 };
 
 struct RouterTile {
@@ -52,7 +66,7 @@ struct RouterCfg {
   static constexpr int A_BYTES = 3 * A_PLANE;
   static constexpr int B_BYTES = RBN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;   // + topk rows (dynamic)
   static constexpr int TMEM_COLS = 2 * RBN <= 256 ? 256 : 512;
   static_assert(RBN % 64 == 0 && RBN <= 256, "RBN");
   static_assert(STAGE_BYTES % 1024 == 0, "alignment");
@@ -71,9 +85,12 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* pfull = empty_bar + STAGES;   // [2] partial buffer written
   uint64_t* pempty = pfull + 2;           // [2] partial buffer drained
   uint64_t* drain_bar = pempty + 2;
-  uint32_t* tmem_holder = (uint32_t*)(drain_bar + 1);
+  uint64_t* epi_bar = drain_bar + 1;      // the 8 epilogue warps meet here (fused selection)
+  uint32_t* tmem_holder = (uint32_t*)(epi_bar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
   int* fills = (int*)(tmem_holder + 2);   // abort cleanup: [0] loads armed, [1] loads consumed
+  volatile int* last_flag = (volatile int*)(fills + 2);   // [2] fused-selection decisions
+  float* topk_rows = (float*)(smem + C::SMEM_BYTES - 1024);  // [topk_warps][E] after the control block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tok_tiles = (args.T + RBN - 1) / RBN;
@@ -89,6 +106,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(smem_u32(pempty + b), 8);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    mbar_init(smem_u32(epi_bar), 8);
     *abort_flag = 0;
     fills[0] = fills[1] = 0;
     fence_mbar_init();
@@ -184,6 +202,20 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t g = 0;
     bool ok = true;
+    // Bounded meeting point of the 8 epilogue warps (an mbarrier phase per meeting), so that
+    // a warp that gives up cannot leave the others waiting; it also orders the shared-memory
+    // flags written before it.
+    uint32_t es_phase = 0;
+    auto epi_sync = [&]() -> bool {
+      bool r = true;
+      if (lane == 0) {
+        mbar_arrive(smem_u32(epi_bar));
+        r = mbar_wait(smem_u32(epi_bar), es_phase, args.status, abort_flag);
+      }
+      es_phase ^= 1u;
+      __syncwarp();
+      return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+    };
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       const RouterTile rt = router_tile(args, RBN, t);
       const int mt = rt.mt, row0 = rt.row0;
@@ -218,8 +250,8 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (!ok) break;
       const int e = mt * 128 + q * 32 + lane;
+      const bool split = args.ksplit > 1;
       if (e < args.E) {
-        const bool split = args.ksplit > 1;
         const float bias = (!split && args.bias) ? __ldg(args.bias + e) : 0.0f;
         float* out = split ? args.zpart + (size_t)rt.split * args.T * args.E : args.z;
 #pragma unroll
@@ -229,6 +261,48 @@ __global__ void __launch_bounds__(320, 1)
             const int n = (cs * MYCH + i) * 16 + j;
             if (n < n_valid) out[(size_t)(row0 + n) * args.E + e] = split ? accv[i][j] : accv[i][j] + bias;
           }
+      }
+
+      // ---- fused selection (see the file comment)
+      const int tt = row0 / RBN;
+      __threadfence();                                 // this thread's stores, before the count
+      if (!(ok = epi_sync())) break;
+      if (warp == 2 && lane == 0) {
+        int last = 1;
+        if (split) {
+          int* c = args.cnt_split + (size_t)tt * args.m_tiles + mt;
+          last = atomicAdd(c, 1) == args.ksplit - 1;
+        }
+        last_flag[0] = last;
+      }
+      if (!(ok = epi_sync())) break;
+      if (!last_flag[0]) continue;
+      __threadfence();                                 // every split of this tile is visible
+      if (split && e < args.E) {
+        // z = the partials summed in split order, plus the logit bias
+        const float bias = args.bias ? __ldg(args.bias + e) : 0.0f;
+        for (int n = cs * (RBN / 2); n < min(n_valid, (cs + 1) * (RBN / 2)); ++n) {
+          const size_t o = (size_t)(row0 + n) * args.E + e;
+          float v = __ldcg(args.zpart + o);
+          for (int sp = 1; sp < args.ksplit; ++sp) v += __ldcg(args.zpart + (size_t)sp * args.T * args.E + o);
+          if (args.bias) v += bias;
+          args.z[o] = v;
+        }
+      }
+      __threadfence();
+      if (!(ok = epi_sync())) break;
+      if (warp == 2 && lane == 0) last_flag[1] = atomicAdd(args.cnt_tile + tt, 1) == args.m_tiles - 1;
+      if (!(ok = epi_sync())) break;
+      if (!last_flag[1]) continue;
+      __threadfence();                                 // every logit of the token tile is visible
+      const int ew = warp - 2;
+      if (ew < args.topk_warps) {
+        float* row = topk_rows + (size_t)ew * args.E;
+        for (int n = ew; n < n_valid; n += args.topk_warps) {
+          const size_t t_ = (size_t)(row0 + n);
+          topk_sigmoid_row(args.z + t_ * args.E, args.sel_bias, args.E, args.k, row, args.idx + t_ * args.k,
+                           args.w + t_ * args.k, lane);
+        }
       }
     }
   }

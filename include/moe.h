@@ -136,13 +136,52 @@ moe_status_t moe_quant_mxfp8(const void* x_bf16, int rows, int cols, uint8_t* q_
  * z = x . W_r + bias (fp32-accurate: W_r is split into three bf16 terms on the tensor
  * cores), s = sigmoid(z); per token the k largest z in descending order (lower expert
  * index on ties) and w_j = s_j / sum of the selected s.  With MOE_BIAS_SELECT_ONLY the
- * bias enters only the selection key z + b (see moe_bias_mode_t).
+ * bias enters only the selection key z + b (see moe_bias_mode_t).  One kernel (plus the
+ * fp32 -> three-plane split of W_r, see MOE_FLAG_STATIC_ROUTER, and a memset of the
+ * selection counters): the CTA that completes a token tile's last logit tile selects
+ * its tokens' experts (a warp per token).
  * x_bf16: device [T][d]; W_r: device fp32 [d][E]; bias: device fp32 [E] or NULL;
  * idx: device int32 [T][k]; w: device fp32 [T][k]; logits_opt: device fp32 [T][E] or
  * NULL (receives z).  Uses the plan workspace. */
 moe_status_t moe_route(moe_plan_t plan, const void* x_bf16, int T, const float* W_r,
                        const float* bias, int32_t* idx, float* w, float* logits_opt,
                        void* stream);
+
+/* ---- Quantile Balancing inputs and hook ----------------------------------------------
+ * Source: "Kimi K3.1 Pro vs gpt-oss-120b" and "Gemma 4 31B vs Kimi K3" (archdiff),
+ * component tables, router row: each expert's selection bias is set every step from a
+ * quantile of routing margins; "Kimi K3, previewed" (embedl blog), "Stable LatentMoE"
+ * section: allocation derived from router-score quantiles.  The update rule itself is not
+ * published, so the library computes what such a rule reads and hands it to the caller's.
+ * Reading: the routing margin of expert e for token t is m[t][e] = key[t][e] - key_(k)(t),
+ * the expert's selection key minus the token's k-th largest key (the top-k threshold;
+ * selected experts have m >= 0), key = z or, with a select-only bias, z + b, all in fp32.
+ * The level-q quantile of expert e is the order statistic of rank clamp(ceil(q T), 1, T)
+ * (1-based, ascending) of m[0..T)[e], rank computed in double on the host.
+ *
+ * moe_route_margin_quantiles: logits: device fp32 [T][E] (moe_route's logits_opt, i.e. z
+ * without a select-only bias); select_bias: device fp32 [E] or NULL (NULL: key = z);
+ * levels: host double [n_levels], each in [0, 1]; quantiles: device fp32 [n_levels][E],
+ * row i for levels[i].  1 <= n_levels <= 16, 1 <= T <= T_max.  Exact (selection, no
+ * interpolation).  Two kernels on `stream`, no host synchronisation; uses the plan's
+ * workspace (the k-th keys), so calls on one plan are ordered on one stream. */
+moe_status_t moe_route_margin_quantiles(moe_plan_t plan, const float* logits, const float* select_bias,
+                                        int T, const double* levels, int n_levels, float* quantiles,
+                                        void* stream);
+/* The caller's bias-update rule.  Called on the calling host thread, after the quantile
+ * kernels were enqueued on `stream` (and before they ran): it must enqueue its own device
+ * work on that stream.  quantiles: device fp32 [n_levels][E] (plan workspace, valid until
+ * the next call on the plan); bias: device fp32 [E], the bias of this step; bias_next:
+ * device fp32 [E] to receive the next step's bias; user: passed through. */
+typedef void (*moe_bias_rule_t)(const float* quantiles, int n_levels, int E, const float* bias,
+                                float* bias_next, void* stream, void* user);
+/* moe_quantile_balance: margin quantiles of this step's routing, then rule(...).  The key
+ * is z + bias under MOE_BIAS_SELECT_ONLY and z under MOE_BIAS_LOGIT (the bias is already in
+ * z); logits as for moe_route_margin_quantiles.  The rule is the caller's: the library
+ * does no arithmetic on the bias itself. */
+moe_status_t moe_quantile_balance(moe_plan_t plan, const float* logits, const float* bias, int T,
+                                  const double* levels, int n_levels, moe_bias_rule_t rule, void* user,
+                                  float* bias_next, void* stream);
 
 /* ---- a4: grouping by expert -----------------------------------------------------------
  * counts[e] = assignments to expert e; offsets = exclusive prefix sum (offsets[E] = T*k);
@@ -236,15 +275,18 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  * MOE_OPT_PREFETCH_DIST: the routed grouped GEMMs prefetch their weight tiles into L2
  *   this many K tiles ahead of the shared-memory loads (0..64, 0 = off).
  * MOE_OPT_PREFETCH_B: accepted and ignored (reserved).
- * MOE_OPT_TILE_N: token rows per grouped-GEMM tile.  0 (default) picks per call: 32 rows
- *   (5-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure weight
- *   stream, else 160 rows (4 stages).  32 or 160 forces one configuration; any other
- *   value is MOE_ERR_INVALID_ARG.  Results do not depend on it beyond fp32 summation
- *   order, which is the same (the K loop runs in the same order in both).
+ * MOE_OPT_TILE_N: token rows per routed grouped-GEMM tile.  0 (default) picks per call:
+ *   128 rows when T*k <= 96*E (most experts within one tile), with the token rows on the
+ *   MMA's M side and 256 weight rows on its N side; else 176 rows with the weights on M
+ *   and the tokens on N.  32 selects a third configuration (weights on M, 32 token rows,
+ *   5-stage pipeline).  32, 128 or 176 forces one configuration; any other value is
+ *   MOE_ERR_INVALID_ARG.  The dense shared-expert GEMMs use 32-row tiles when T*k <= 8*E
+ *   and 176 otherwise.  Results agree within fp32 accumulation (the K loop runs in the same
+ *   order in all three).
  * MOE_OPT_ROUTER_SPLIT (read only): the number of K splits the last moe_route used for
  *   the router GEMM (1 = none).  With few tokens the router splits d over up to one
- *   CTA per SM and adds the fp32 partials in split order (plus the bias) in one more
- *   kernel, so that call launches 4 kernels instead of 3.
+ *   CTA per SM; the CTA that finishes a tile's last split adds the fp32 partials in split
+ *   order (plus the bias) inside the same kernel.
  * MOE_OPT_SHARED_SPLIT / MOE_OPT_SHARED_SPLIT_DOWN (read only): K splits of the shared
  *   expert's gate/up and down GEMMs in the last moe_forward (1 = none; 0 without a shared
  *   expert).  With few tokens these dense GEMMs split K over the SMs.  Each split GEMM writes
@@ -266,8 +308,8 @@ moe_status_t moe_plan_get_option(moe_plan_t plan, int option, int* value);
  * n >= MOE_NUM_STAGES entries; `launches` may be NULL), then forgets them. */
 enum {
   MOE_STAGE_ROUTER_SPLIT = 0,    /* W_r -> three bf16 planes */
-  MOE_STAGE_ROUTER_GEMM = 1,     /* logits on the tensor cores */
-  MOE_STAGE_TOPK = 2,            /* sigmoid top-k + renormalise */
+  MOE_STAGE_ROUTER_GEMM = 1,     /* logits on the tensor cores + fused sigmoid top-k */
+  MOE_STAGE_TOPK = 2,            /* (sigmoid top-k is fused into the router kernel: unused) */
   MOE_STAGE_PERMUTE = 3,         /* histogram, scan, placement (3 kernels) */
   MOE_STAGE_QUANT = 4,           /* MXFP8 quantise + scatter to expert order */
   MOE_STAGE_GATE_UP = 5,         /* routed gate/up GEMM + GLU + MXFP8 requant */
@@ -285,8 +327,8 @@ moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n)
 /* ---- introspection (tests) ----------------------------------------------------------
  * Device pointer and size of a workspace buffer after a call, for checking the steps:
  *   0 xq  E4M3 [T*k][d] activations in expert order
- *   1 xs  scales of xq, tile-major: for group-tile g (tiles of <= 160 rows per expert,
- *         ceil(count/160) tiles of round16(ceil(count/tiles)) rows each, numbered in
+ *   1 xs  scales of xq, tile-major: for group-tile g (tiles of <= 176 rows per expert,
+ *         ceil(count/176) tiles of round16(ceil(count/tiles)) rows each, numbered in
  *         expert order) and 128-column K tile kt, 1 KB at (g*(d/128) + kt)*1024; row n of
  *         the tile, 32-block j of the K tile at (n/128)*512 + (n%32)*16 + ((n%128)/32)*4 + j
  *   2 hq  E4M3 [T*k][I] GLU output in expert order
@@ -294,6 +336,7 @@ moe_status_t moe_plan_stage_ms(moe_plan_t plan, float* ms, int* launches, int n)
  *   4 O   bf16 [T*k][d] expert outputs in expert order
  *   5 ys  fp32 [T][d] shared expert output
  *   6 logits fp32 [T][E]
+ *   7 quantiles fp32 [16][E]: the buffer moe_quantile_balance hands to the bias rule
  * Row counts use the T of the last call. */
 moe_status_t moe_debug_buffer(moe_plan_t plan, int which, void** dev_ptr, size_t* bytes);
 

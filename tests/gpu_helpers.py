@@ -47,7 +47,7 @@ def unpack_expert_codes(ex, e, d, I):
     }
 
 
-def decode_tile_major_scales(buf, counts, k_tiles, bn=160):
+def decode_tile_major_scales(buf, counts, k_tiles, bn=176):
     """Token-side scale bytes [A][k_tiles*4] from the tile-major layout documented in
     include/moe.h (debug buffers 1 and 3), using the expert row counts."""
     buf = np.asarray(buf, dtype=np.uint8)

@@ -1,13 +1,23 @@
 """GPU parity at the full Kimi-K3 shapes (d=7168, 896 experts, top-16, I=3072, one bf16
 shared expert), in the launch configuration the benchmark times.
 
-Checked on every token: router logits against fp64 (sampled rows), bit-exact top-k on
-the GPU's own logits (all rows), bit-exact permutation and MXFP8 bytes (all rows), finite
-outputs.  Checked on sampled tokens: the layer output against the fp64 oracle (the
-oracle quantises each touched expert's fp32 masters itself, in a process pool)."""
-import multiprocessing as mp
-import os
+Every Kimi-K3 workload of the specification is covered:
+  * decode, T=64 (seed 1): the layer output of every token against the fp64 oracle;
+  * prefill, T=8192 (seed 2): 64 tokens chosen to touch at least 256 experts (among them
+    the most loaded ones), plus the GLU output (MXFP8 codes and scales) and the expert
+    outputs of whole experts, in both GEMM orientations (176-row tiles with the weights on
+    the MMA's M side, the default here; 128-row tiles with the tokens on M, where every
+    expert spans two tiles);
+  * skewed prefill, T=32768 (seed 3): 64 tokens, among them tokens of the hottest experts,
+    whose thousands of rows span many tiles;
+  * token-count sweep (seed 4): T = 1, 16, 256 (every token) and 2048, 16384 (32 sampled
+    tokens each).
+On every token of every run: router logits against fp64 (sampled rows), bit-exact top-k on
+the GPU's own logits, bit-exact permutation, bit-exact MXFP8 activations, finite outputs.
 
+The oracle quantises each touched expert's fp32 masters itself, in a process pool
+(tests/k3_oracle.py); its routing comes from fp64 logits.  Tokens whose 16th/17th score gap
+is below 1e-6 are counted and excluded from the error statistics."""
 import numpy as np
 import pytest
 import torch
@@ -15,98 +25,12 @@ import torch
 from block_scaled_moe_sigmoid_b200 import api, synth
 from oracle import layer, mx, permute as operm, router
 
-from .gpu_helpers import layer_stats
+from . import k3_oracle
+from .gpu_helpers import decode_tile_major_scales, layer_stats
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 MAX_REL, MEAN_REL = 2e-2, 2e-3
-
-
-class K3Case:
-    def __init__(self, wl, T):
-        self.wl, self.T = wl, T
-        self.x = synth.draw_x(wl, T, device="cuda")
-        self.W_r, self.bias = synth.draw_router(wl, device="cuda")
-        self.plan = api.Plan(T, wl.d, wl.E, wl.k, wl.I, wl.I_shared)
-        self.experts = api.Experts(wl.d, wl.I, wl.E)
-        for e in range(wl.E):
-            self.experts.pack(e, *synth.draw_expert(wl, e, device="cuda"))
-        self.shared = api.Shared(wl.d, wl.I_shared)
-        self.shared_w = synth.draw_shared(wl, device="cuda")
-        self.shared.pack(*self.shared_w)
-        torch.cuda.synchronize()
-
-    def run(self):
-        wl, T = self.wl, self.T
-        self.logits = torch.empty((T, wl.E), dtype=torch.float32, device="cuda")
-        self.idx, self.w = self.plan.route(self.x, self.W_r, self.bias, logits=self.logits)
-        self.y = self.plan.forward(self.x, self.idx, self.w, self.experts, self.shared)
-        code, bits = self.plan.check()
-        assert code == 0, (code, bits)
-
-    def free(self):
-        for name in ("experts", "shared", "plan", "x", "logits", "y"):
-            if hasattr(self, name):
-                delattr(self, name)
-        torch.cuda.empty_cache()
-
-
-def _check(case, sample_tokens, logit_rows=64):
-    wl, T = case.wl, case.T
-    case.run()
-    x = case.x.float().cpu().numpy().astype(np.float64)
-    z_gpu = case.logits.cpu().numpy().astype(np.float64)
-    idx = case.idx.cpu().numpy()
-    w = case.w.cpu().numpy()
-    y = case.y.float().cpu().numpy().astype(np.float64)
-    assert np.all(np.isfinite(y))
-
-    # router: fp64 logits on sampled rows; bit-exact top-k on the GPU logits for every row
-    W_r, bias = case.W_r.cpu().numpy(), case.bias.cpu().numpy()
-    g = np.random.default_rng(T)
-    rows = np.unique(np.concatenate([g.choice(T, size=min(logit_rows, T), replace=False), sample_tokens]))
-    z_ref = router.router_logits(x[rows], W_r, bias)
-    assert np.max(np.abs(z_gpu[rows] - z_ref)) < 5e-5
-    idx_g, w_g, _ = router.route(z_gpu, wl.k)
-    assert np.array_equal(idx, idx_g)
-    assert np.allclose(w, w_g, rtol=2e-6, atol=1e-7)
-    idx_o, w_o, gap = router.route(z_ref, wl.k)
-    assert not np.any(np.any(idx[rows] != idx_o, axis=1) & (gap >= 1e-6))
-
-    # permutation (bit-exact, every assignment) and the MXFP8 activations in expert order
-    counts, offsets, perm_tok, inv = case.plan.permute(case.idx)
-    c_ref, o_ref, p_ref, i_ref = operm.permute(idx, wl.E)
-    assert np.array_equal(counts.cpu().numpy(), c_ref) and np.array_equal(offsets.cpu().numpy(), o_ref)
-    assert np.array_equal(perm_tok.cpu().numpy(), p_ref) and np.array_equal(inv.cpu().numpy(), i_ref)
-    qrows = rows if T > 8192 else np.arange(T)          # every row up to the prefill size
-    xq_ref, xs_ref = mx.quantize_mx(x[qrows], "e4m3")
-    q_gpu, s_gpu = api.moe_quant_mxfp8(case.x)
-    assert np.array_equal(q_gpu.cpu().numpy()[qrows], xq_ref)
-    assert np.array_equal(s_gpu.cpu().numpy()[qrows], xs_ref)
-    # the forward pass's own copy in expert order (first row of each sampled token's slots)
-    xq_perm = case.plan.debug_tensor(0, torch.uint8, (T * wl.k, wl.d))
-    for t in sample_tokens:
-        pos = i_ref[t]
-        ref_q, _ = mx.quantize_mx(x[t:t + 1], "e4m3")
-        assert np.array_equal(xq_perm[torch.as_tensor(pos, device="cuda").long()].cpu().numpy(),
-                              np.repeat(ref_q, len(pos), axis=0))
-
-    # layer output on the sampled tokens
-    st_rows = np.asarray(sample_tokens)
-    need = sorted(set(int(e) for e in idx_o[np.searchsorted(rows, st_rows)].ravel()))
-    masters = {e: tuple(t.cpu().numpy() for t in synth.draw_expert(wl, e, device="cuda")) for e in need}
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(min(8, os.cpu_count() or 1)) as pool:
-        quant = dict(zip(need, pool.starmap(layer.quantize_expert, [masters[e] for e in need])))
-    del masters
-    shared = tuple(t.float().cpu().numpy().astype(np.float64) for t in case.shared_w)
-    y_ref = layer.moe_layer(x[st_rows], idx_o[np.searchsorted(rows, st_rows)],
-                            w_o[np.searchsorted(rows, st_rows)],
-                            lambda e: layer.decode_expert(quant[e]), shared)
-    st = layer_stats(y[st_rows], y_ref, gap[np.searchsorted(rows, st_rows)])
-    print(wl.name, T, st)
-    assert st["max_rel"] <= MAX_REL and st["mean_rel"] <= MEAN_REL, st
-    return st
 
 
 @pytest.fixture(autouse=True)
@@ -115,30 +39,237 @@ def _cuda():
         pytest.skip("needs a CUDA GPU")
 
 
-def test_k3_decode_t64():
-    case = K3Case(synth.WORKLOADS["k3_decode_t64"], 64)
-    try:
-        _check(case, sample_tokens=[5, 63])
-    finally:
-        case.free()
+class K3Experts:
+    """The workload's 896 experts, packed once (31.4 GB), and its shared expert."""
+
+    def __init__(self, wl):
+        self.wl = wl
+        self.experts = api.Experts(wl.d, wl.I, wl.E)
+        for e in range(wl.E):
+            self.experts.pack(e, *synth.draw_expert(wl, e, device="cuda"))
+        self.shared = api.Shared(wl.d, wl.I_shared)
+        self.shared_w = synth.draw_shared(wl, device="cuda")
+        self.shared.pack(*self.shared_w)
+        torch.cuda.synchronize()
+
+    def oracle_shared(self):
+        return tuple(t.float().cpu().numpy().astype(np.float64) for t in self.shared_w)
 
 
-def test_k3_prefill_t8192():
-    case = K3Case(synth.WORKLOADS["k3_prefill_t8192"], 8192)
-    try:
-        _check(case, sample_tokens=[0, 8191])
-    finally:
-        case.free()
+class K3Run:
+    """One batch of T tokens through moe_route + moe_forward."""
+
+    def __init__(self, ex, T):
+        wl = ex.wl
+        self.ex, self.wl, self.T = ex, wl, T
+        self.x = synth.draw_x(wl, T, device="cuda")
+        self.W_r, self.bias = synth.draw_router(wl, device="cuda")
+        self.plan = api.Plan(T, wl.d, wl.E, wl.k, wl.I, wl.I_shared)
+
+    def run(self, tile_n=0):
+        wl, T = self.wl, self.T
+        api.moe_plan_set_option(self.plan.handle, api.MOE_OPT_TILE_N, tile_n)
+        self.logits = torch.empty((T, wl.E), dtype=torch.float32, device="cuda")
+        self.idx, self.w = self.plan.route(self.x, self.W_r, self.bias, logits=self.logits)
+        self.y = self.plan.forward(self.x, self.idx, self.w, self.ex.experts, self.ex.shared)
+        code, bits = self.plan.check()
+        assert code == 0, (code, bits)
+        return self.y.float().cpu().numpy().astype(np.float64)
+
+    def check_routing_and_grouping(self, logit_rows):
+        """Everything except the layer output; returns the oracle's fp64 routing."""
+        wl, T = self.wl, self.T
+        x = self.x.float().cpu().numpy().astype(np.float64)
+        z_gpu = self.logits.cpu().numpy().astype(np.float64)
+        idx = self.idx.cpu().numpy()
+        w = self.w.cpu().numpy()
+        assert np.all(np.isfinite(self.y.float().cpu().numpy()))
+        W_r, bias = self.W_r.cpu().numpy(), self.bias.cpu().numpy()
+        # fp64 logits (sampled rows) and the oracle's own routing of every token
+        z_ref = router.router_logits(x, W_r, bias)
+        assert np.max(np.abs(z_gpu[logit_rows] - z_ref[logit_rows])) < 5e-5
+        idx_o, w_o, gap = router.route(z_ref, wl.k)
+        # bit-exact selection given the GPU's own logits, every row
+        idx_g, w_g, _ = router.route(z_gpu, wl.k)
+        assert np.array_equal(idx, idx_g)
+        assert np.allclose(w, w_g, rtol=2e-6, atol=1e-7)
+        # against the fp64 routing: the selected set may differ only where the fp64 logit
+        # gap between the token's k-th and (k+1)-th expert is within twice the GPU's logit
+        # error on that token (fp32 logits may order the two the other way).  The order
+        # inside the set may differ the same way between adjacent experts; the layer output
+        # does not depend on it.
+        self.match = np.all(np.sort(idx, axis=1) == np.sort(idx_o, axis=1), axis=1)
+        reordered = int(np.sum(self.match & np.any(idx != idx_o, axis=1)))
+        if reordered:
+            print(f"T={T}: {reordered} tokens select the same set in another order")
+        if not np.all(self.match):
+            bad = np.flatnonzero(~self.match)
+            zs = -np.sort(-z_ref[bad], axis=1)
+            logit_gap = zs[:, wl.k - 1] - zs[:, wl.k]
+            err = np.max(np.abs(z_gpu[bad] - z_ref[bad]), axis=1)
+            assert np.all(logit_gap <= 2 * err), (bad, logit_gap, err)
+            print(f"T={T}: {len(bad)} tokens route differently from fp64 (logit gap within "
+                  f"the fp32 error), their gaps {gap[bad]}")
+        # permutation (bit-exact, every assignment) and the MXFP8 activations
+        counts, offsets, perm_tok, inv = self.plan.permute(self.idx)
+        ref = operm.permute(idx, wl.E)
+        for got, r in zip((counts, offsets, perm_tok, inv), ref):
+            assert np.array_equal(got.cpu().numpy(), r)
+        q_gpu, s_gpu = api.moe_quant_mxfp8(self.x)
+        xq_ref, xs_ref = mx.quantize_mx(x, "e4m3")
+        assert np.array_equal(q_gpu.cpu().numpy(), xq_ref) and np.array_equal(s_gpu.cpu().numpy(), xs_ref)
+        return x, idx_o, w_o, gap, ref
 
 
-def test_k3_skewed_t32768():
+def _pick_tokens(idx, n, min_experts, first=(), prefer=None):
+    """n tokens: `first`, then greedy picks.  While fewer than min_experts experts are
+    covered, each pick adds the most new experts; afterwards the fewest (so the oracle
+    quantises as few experts as the coverage allows).  `prefer`: experts counted as covered
+    from the start (already needed elsewhere)."""
+    T, k = idx.shape
+    E = max(int(idx.max()) + 1, 0 if prefer is None else len(prefer))
+    chosen = list(dict.fromkeys(int(t) for t in first))[:n]
+    covered = np.zeros(E, bool) if prefer is None else prefer.copy()
+    covered[idx[chosen].ravel()] = True
+    free = np.ones(T, bool)
+    free[chosen] = False
+    while len(chosen) < min(n, T):
+        new = (~covered[idx]).sum(axis=1)
+        new = np.where(free, new, -1 if covered.sum() < min_experts else k + 1)
+        t = int(np.argmax(new) if covered.sum() < min_experts else np.argmin(new))
+        chosen.append(t)
+        free[t] = False
+        covered[idx[t]] = True
+    return np.array(sorted(chosen))
+
+
+def _stats(name, y_gpu, y_ref, gap, match):
+    """Error statistics (reading R17) over the tokens whose routing matches the fp64
+    routing and whose k/k+1 score gap is >= 1e-6; the others are counted."""
+    st = layer_stats(y_gpu[match], y_ref[match], gap[match])
+    st["routing_differs"] = int((~match).sum())
+    print(name, st)
+    assert st["max_rel"] <= MAX_REL and st["mean_rel"] <= MEAN_REL, (name, st)
+    return st
+
+
+def test_k3_decode_t64_every_token():
+    wl = synth.WORKLOADS["k3_decode_t64"]
+    ex = K3Experts(wl)
+    r = K3Run(ex, wl.T)
+    y = r.run()
+    x, idx_o, w_o, gap, _ = r.check_routing_and_grouping(np.arange(wl.T))
+    y_ref, _ = k3_oracle.layer_outputs(wl, x, idx_o, w_o, ex.oracle_shared())
+    _stats("k3_decode_t64 all 64 tokens", y, y_ref, gap, r.match)
+
+
+def _stage_expert_checks(r, e_list, perm, extra, bn):
+    """GLU output (MXFP8 codes + scales) and expert outputs of whole experts, expert order."""
+    wl = r.wl
+    A = r.T * wl.k
+    counts, offsets, perm_tok, _ = perm
+    hq = r.plan.debug_tensor(2, torch.uint8, (A, wl.I)).cpu().numpy()
+    _, nbytes = api.moe_debug_buffer(r.plan.handle, 3)
+    hs = decode_tile_major_scales(r.plan.debug_tensor(3, torch.uint8, (nbytes,)).cpu().numpy(),
+                                  counts, wl.I // 128, bn)
+    O = r.plan.debug_tensor(4, torch.bfloat16, (A, wl.d)).float().cpu().numpy()
+    for e in e_list:
+        rows = np.arange(offsets[e], offsets[e + 1])
+        o_ref, _, hq_ref, hs_ref = extra[e]
+        H = mx.dequantize_mx(hq[rows], hs[rows], "e4m3")
+        H_ref = mx.dequantize_mx(hq_ref, hs_ref, "e4m3")
+        diff = np.abs(H - H_ref)
+        scale = np.repeat(mx.e8m0_value(hs_ref), 32, axis=1)
+        worst = float(np.max(diff / (np.abs(H_ref) + scale * 2.0 ** -9)))
+        mism = int(np.sum(diff > 0))
+        assert worst <= 0.13, (e, bn, worst)                # at most one E4M3 step
+        assert mism <= 0.01 * H.size, (e, bn, mism)
+        rel = np.linalg.norm(O[rows] - o_ref, axis=1) / np.linalg.norm(o_ref, axis=1)
+        assert rel.max() < 1e-2, (e, bn, rel.max())
+        print(f"expert {e}: {len(rows)} rows, tile rows {bn}: GLU codes differing {mism}, "
+              f"worst {worst:.3g}; expert output normwise max {rel.max():.3g}")
+
+
+def test_k3_prefill_t8192_sampled_tokens_and_whole_experts():
+    wl = synth.WORKLOADS["k3_prefill_t8192"]
+    ex = K3Experts(wl)
+    r = K3Run(ex, wl.T)
+    y_big = r.run(tile_n=0)
+    bn_big = api.moe_plan_get_option(r.plan.handle, api.MOE_OPT_TILE_N)
+    g = np.random.default_rng(wl.T)
+    x, idx_o, w_o, gap, perm = r.check_routing_and_grouping(g.choice(wl.T, 64, replace=False))
+    counts = perm[0]
+    order = np.argsort(-counts, kind="stable")
+    # whole experts for the stage checks: the two most loaded (rows over several tiles),
+    # a median one and the least loaded non-empty one
+    nz = order[counts[order] > 0]
+    e_stage = [int(nz[0]), int(nz[1]), int(nz[len(nz) // 2]), int(nz[-1])]
+    hot_tokens = [int(np.argwhere(idx_o == e)[0, 0]) for e in e_stage[:2]]
+    tokens = _pick_tokens(idx_o, 64, 256, first=hot_tokens + [0, wl.T - 1])
+    assert len(np.unique(idx_o[tokens])) >= 256
+    X = mx.dequantize_mx(*mx.quantize_mx(x, "e4m3"), "e4m3")
+    perm_tok, offs = perm[2], perm[1]
+    blocks = {e: X[perm_tok[offs[e]:offs[e + 1]]] for e in e_stage}
+    y_ref, extra = k3_oracle.layer_outputs(wl, x[tokens], idx_o[tokens], w_o[tokens], ex.oracle_shared(),
+                                           stage_experts=set(e_stage), extra_rows=blocks)
+    print("experts touched by the sampled tokens:", len(np.unique(idx_o[tokens])))
+    _stats(f"k3_prefill_t8192 64 tokens, tile rows {bn_big}", y_big[tokens], y_ref, gap[tokens], r.match[tokens])
+    _stage_expert_checks(r, e_stage, perm, extra, bn_big)
+    # the other orientation (token rows on the MMA's M side, <= 128 rows per tile: every
+    # expert here spans two tiles): same routing, same oracle outputs
+    y_wn = r.run(tile_n=128)
+    assert api.moe_plan_get_option(r.plan.handle, api.MOE_OPT_TILE_N) == 128
+    _stats("k3_prefill_t8192 64 tokens, tile rows 128", y_wn[tokens], y_ref, gap[tokens], r.match[tokens])
+    _stage_expert_checks(r, e_stage, perm, extra, 128)
+
+
+def test_k3_skewed_t32768_sampled_tokens():
     """Zipf-like logit bias: hot experts get thousands of rows (many GEMM tiles each)."""
     wl = synth.WORKLOADS["k3_skewed_t32768"]
-    case = K3Case(wl, 32768)
-    try:
-        st = _check(case, sample_tokens=[12345], logit_rows=32)
-        counts = np.bincount(case.idx.cpu().numpy().ravel(), minlength=wl.E)
-        assert counts.max() > 5 * counts.mean()       # the load really is skewed
-        print("skewed load: max", counts.max(), "experts used", int((counts > 0).sum()))
-    finally:
-        case.free()
+    ex = K3Experts(wl)
+    r = K3Run(ex, wl.T)
+    y = r.run()
+    g = np.random.default_rng(wl.T)
+    x, idx_o, w_o, gap, perm = r.check_routing_and_grouping(g.choice(wl.T, 32, replace=False))
+    counts = perm[0]
+    assert counts.max() > 5 * counts.mean()           # the load really is skewed
+    hot = np.argsort(-counts, kind="stable")[:8]
+    hot_tokens = [int(np.argwhere(idx_o == e)[-1, 0]) for e in hot]
+    # the routing uses only a few hundred experts in all (Zipf-like bias): the sample
+    # covers the hottest and at least 160 distinct ones
+    tokens = _pick_tokens(idx_o, 64, 160, first=hot_tokens + [12345])
+    y_ref, _ = k3_oracle.layer_outputs(wl, x[tokens], idx_o[tokens], w_o[tokens], ex.oracle_shared())
+    print("skewed load: max", counts.max(), "experts used", int((counts > 0).sum()),
+          "experts touched by the sampled tokens", len(np.unique(idx_o[tokens])))
+    _stats("k3_skewed_t32768 64 tokens", y[tokens], y_ref, gap[tokens], r.match[tokens])
+
+
+def test_k3_token_count_sweep():
+    """configs: T in {1, 16, 256, 2048, 16384}, seed 4; every token up to T=256, 32
+    sampled tokens above.  The experts are packed once and one oracle pass serves all T."""
+    wl = synth.WORKLOADS["k3_sweep"]
+    ex = K3Experts(wl)
+    parts = []
+    covered = np.zeros(wl.E, bool)
+    for T in wl.sweep:
+        r = K3Run(ex, T)
+        y = r.run()
+        g = np.random.default_rng(T)
+        rows = np.arange(T) if T <= 256 else g.choice(T, 4, replace=False)
+        x, idx_o, w_o, gap, _ = r.check_routing_and_grouping(rows if T > 256 else np.arange(T))
+        # above T=256: 4 random tokens, then tokens whose experts the earlier T (every token
+        # of T=256 touches nearly all 896) already need, so the oracle's expert set grows little
+        tokens = rows if T <= 256 else _pick_tokens(idx_o, 32, 0, first=rows, prefer=covered)
+        covered[idx_o[tokens].ravel()] = True
+        parts.append((T, y[tokens], x[tokens], idx_o[tokens], w_o[tokens], gap[tokens],
+                      api.moe_plan_get_option(r.plan.handle, api.MOE_OPT_TILE_N), r.match[tokens]))
+        del r
+        torch.cuda.empty_cache()
+    y_ref, _ = k3_oracle.layer_outputs(wl, np.concatenate([p[2] for p in parts]),
+                                       np.concatenate([p[3] for p in parts]),
+                                       np.concatenate([p[4] for p in parts]), ex.oracle_shared())
+    o = 0
+    for T, y, _, idx_o, _, gap, bn, match in parts:
+        n = len(y)
+        _stats(f"k3_sweep T={T} ({n} tokens, tile rows {bn})", y, y_ref[o:o + n], gap, match)
+        o += n
