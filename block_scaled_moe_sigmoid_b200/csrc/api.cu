@@ -18,17 +18,18 @@ using namespace moe;
 
 namespace {
 
-// Routed grouped-GEMM tile configurations:
-//   WN (gemm.cuh): token rows on the MMA's M side, 256 weight rows on N, up to 128 token
-//   rows per tile, 4-stage smem ring (50 KB stages).  Each K block is one M=128 x N=256
-//   MMA whatever the token count, instead of two M=128 x N=n ones: the default while most
-//   experts have at most 128 rows (T*k <= 96*E), decode included;
-//   large: swap-AB (256 weight rows on M, up to 176 token rows on N), 4 stages (56 KB).
-//   Kimi-K3 prefill (T=8192) gives an expert ~146 +- 12 rows, so 176 keeps all but a
-//   handful of experts in one tile (with 160, one in eight was split in two half-full
-//   tiles, each costing as much tensor time as a full one);
-//   small: swap-AB with up to 32 token rows, 5 stages (38 KB): selectable, and the dense
-//   shared-expert GEMMs' tile for a few tokens per expert.
+// Routed grouped-GEMM tile configurations (token rows per tile), chosen per call:
+//   176 (default when T*k > 8*E): swap-AB, 256 weight rows on the MMA's M side and up to
+//   176 token rows on N, 4-stage smem ring (56 KB stages).  Kimi-K3 prefill (T=8192) gives
+//   an expert ~146 +- 12 rows, so 176 keeps all but a handful of experts in one tile (with
+//   160, one in eight was split in two half-full tiles, each costing as much tensor time as
+//   a full one);
+//   32 (default when T*k <= 8*E, decode): swap-AB with up to 32 token rows, 5 stages
+//   (38 KB): with a few tokens per expert the weight stream is the whole cost and the fifth
+//   stage keeps another 16 KB weight tile per SM in flight;
+//   128 (selectable): the WN orientation (gemm.cuh), token rows on M and 256 weight rows on
+//   N, 4 stages (50 KB).  Half the MMAs of swap-AB per weight byte, bit-identical results,
+//   but measured slower at every token count (see the design notes), so never the default.
 constexpr int kBN = 176, kStages = 4;
 constexpr int kBNMid = 128, kStagesMid = 4;
 constexpr int kBNSmall = 32, kStagesSmall = 5;
@@ -144,8 +145,7 @@ struct moe_plan_s {
   // token rows per routed GEMM tile for a call with T tokens
   int tile_rows(int T) const {
     if (tile_n_opt) return tile_n_opt;
-    const long long A = (long long)T * k;
-    return A <= 96ll * E ? kBNMid : kBN;  // WN while most experts fit 128 rows
+    return (long long)T * k <= 8ll * E ? kBNSmall : kBN;   // <= 8 tokens per expert on average
   }
   // token rows per tile of the dense (shared-expert, latent projection) GEMMs
   int dense_rows(int T) const { return (long long)T * k <= 8ll * E ? kBNSmall : kBN; }
@@ -480,9 +480,10 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
-    // the fused selection keeps one E-float row per epilogue warp after the pipeline
-    ra.topk_warps = std::min(8, (kMaxDynSmem - RC::SMEM_BYTES) / (E * 4));
-    if (ra.topk_warps < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+    // the fused selection holds the keys in registers up to E = 1024; beyond, one E-float
+    // shared-memory row per selecting warp after the pipeline
+    ra.topk_warps = E <= 32 * kTopkKeysPerLane ? 0 : std::min(8, (kMaxDynSmem - RC::SMEM_BYTES) / (E * 4));
+    if (E > 32 * kTopkKeysPerLane && ra.topk_warps < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
     const int smem = RC::SMEM_BYTES + ra.topk_warps * E * 4;
     static std::atomic<uint64_t> router_done{0};
     if (ensure_smem_attr(kern, kMaxDynSmem, router_done) != cudaSuccess) return MOE_ERR_CUDA;

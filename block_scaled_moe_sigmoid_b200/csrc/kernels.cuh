@@ -306,14 +306,68 @@ __global__ void perm_place_kernel(const int* __restrict__ idx, int T, int k, int
 }
 
 // ---------------------------------------------------------------- top-k
+// fp32 -> uint32 with the same order (negatives flipped whole, positives' sign bit set).
+__device__ __forceinline__ uint32_t f32_order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float f32_from_order_key(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 // Selection for one token, by one warp: key = z (+ select_bias in the select-only mode,
-// fp32); k rounds of a warp arg-max over the keys (descending value, lower index on equal
-// values), then w_j = s_j / sum of the selected s, s = sigmoid(z).  row: the warp's
-// shared-memory scratch of E floats.  z is read through L2 (__ldcg): it may have been
-// written by other CTAs of the same kernel.
-__device__ __forceinline__ void topk_sigmoid_row(const float* __restrict__ z_row, const float* __restrict__ select_bias,
-                                                 int E, int k, float* row, int* __restrict__ idx_out,
-                                                 float* __restrict__ w_out, int lane) {
+// fp32); the k largest keys in descending order, the lower expert index first among equal
+// keys; then w_j = s_j / sum of the selected s, s = sigmoid(z).  z is read through L2
+// (__ldcg): it may have been written by other CTAs of the same kernel.
+//
+// Fast form (E <= 32 * KPL): each lane keeps the keys of experts lane, lane + 32, ... in
+// registers.  A round takes the lane's first largest key, then the warp's largest as a
+// redux.sync max of an order-preserving uint32 map, then the lowest index among the lanes
+// holding it as a redux.sync min; the owning lane marks that key taken.
+constexpr int kTopkKeysPerLane = 32;
+__device__ __forceinline__ void topk_sigmoid_row_regs(const float* __restrict__ z_row,
+                                                      const float* __restrict__ select_bias, int E, int k,
+                                                      int* __restrict__ idx_out, float* __restrict__ w_out,
+                                                      int lane) {
+  float v[kTopkKeysPerLane];
+#pragma unroll
+  for (int j = 0; j < kTopkKeysPerLane; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? (select_bias ? __ldcg(z_row + e) + __ldg(select_bias + e) : __ldcg(z_row + e)) : -INFINITY;
+  }
+  float ssum = 0.0f, my_s = 0.0f;
+  int my_i = -1;
+  uint32_t taken = 0;   // bit j: key j of this lane already selected (v itself is never rewritten)
+  for (int r = 0; r < k; ++r) {
+    float bv = (taken & 1u) ? -INFINITY : v[0];
+    int bj = 0;
+#pragma unroll
+    for (int j = 1; j < kTopkKeysPerLane; ++j) {
+      const float vj = ((taken >> j) & 1u) ? -INFINITY : v[j];
+      if (vj > bv) { bv = vj; bj = j; }        // ascending index: the first max is kept
+    }
+    const uint32_t bu = f32_order_key(bv + 0.0f);   // -0 -> +0: equal keys compare equal
+    const uint32_t mu = __reduce_max_sync(0xffffffffu, bu);
+    const uint32_t cand = bu == mu ? (uint32_t)(lane + 32 * bj) : 0xffffffffu;
+    const int bi = (int)__reduce_min_sync(0xffffffffu, cand);
+    const float zsel = select_bias ? __ldcg(z_row + bi) : f32_from_order_key(mu);
+    const float s = 1.0f / (1.0f + expf(-zsel));
+    ssum += s;
+    if (lane == r) { my_s = s; my_i = bi; }
+    if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
+  }
+  if (lane < k) {
+    idx_out[lane] = my_i;
+    w_out[lane] = my_s / ssum;
+  }
+  __syncwarp();
+}
+
+// General form (any E): the keys in the warp's shared-memory row of E floats; k rounds of a
+// warp arg-max (shuffles, lower index on equal keys).
+__device__ __forceinline__ void topk_sigmoid_row_smem(const float* __restrict__ z_row, const float* __restrict__ select_bias,
+                                                      int E, int k, float* row, int* __restrict__ idx_out,
+                                                      float* __restrict__ w_out, int lane) {
   for (int e = lane; e < E; e += 32)
     row[e] = select_bias ? __ldcg(z_row + e) + __ldg(select_bias + e) : __ldcg(z_row + e);
   __syncwarp();
@@ -576,15 +630,6 @@ __global__ void kth_key_kernel(const float* __restrict__ z, const float* __restr
     __syncwarp();
   }
   if (lane == 0) theta[t] = bv;
-}
-
-// fp32 -> uint32 with the same order (negatives flipped whole, positives' sign bit set).
-__device__ __forceinline__ uint32_t f32_order_key(float v) {
-  const uint32_t b = __float_as_uint(v);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float f32_from_order_key(uint32_t u) {
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
 // Exact order statistics of the margins by radix select, 8 bits a pass from the top.

@@ -17,7 +17,7 @@
 // Selection is fused: the CTA that completes the last split of a (token tile, expert tile)
 // adds the partials in split order plus the bias and writes z; the CTA that completes the
 // last expert tile of a token tile has every logit of those tokens and runs the sigmoid
-// top-k (topk_sigmoid_row) for them.  "Last" is decided by counters (atomicAdd after a
+// top-k (topk_sigmoid_row_regs, or _smem for E > 1024) for them.  "Last" is decided by counters (atomicAdd after a
 // fence of the CTA's stores); nothing waits on another CTA, and the counters are zeroed
 // before the launch.
 #pragma once
@@ -278,15 +278,41 @@ __global__ void __launch_bounds__(320, 1)
       if (!(ok = epi_sync())) break;
       if (!last_flag[0]) continue;
       __threadfence();                                 // every split of this tile is visible
-      if (split && e < args.E) {
-        // z = the partials summed in split order, plus the logit bias
-        const float bias = args.bias ? __ldg(args.bias + e) : 0.0f;
-        for (int n = cs * (RBN / 2); n < min(n_valid, (cs + 1) * (RBN / 2)); ++n) {
-          const size_t o = (size_t)(row0 + n) * args.E + e;
-          float v = __ldcg(args.zpart + o);
-          for (int sp = 1; sp < args.ksplit; ++sp) v += __ldcg(args.zpart + (size_t)sp * args.T * args.E + o);
-          if (args.bias) v += bias;
-          args.z[o] = v;
+      if (split) {
+        // z = the partials summed in split order, plus the logit bias.  The 256 epilogue
+        // threads walk the tile's (token, expert) elements flat (expert fastest, so a warp's
+        // loads are coalesced), four elements and eight partials at a time in flight.
+        const int et = (warp - 2) * 32 + lane;
+        const int nel = n_valid * 128;
+        const size_t plane = (size_t)args.T * args.E;
+        for (int i0 = et; i0 < nel; i0 += 4 * 256) {
+          size_t o[4];
+          bool in[4];
+          float v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * 256;
+            const int ee = mt * 128 + (i & 127);
+            in[u] = i < nel && ee < args.E;
+            o[u] = in[u] ? (size_t)(row0 + (i >> 7)) * args.E + ee : 0;
+            v[u] = in[u] ? __ldcg(args.zpart + o[u]) : 0.0f;
+          }
+          for (int s0 = 1; s0 < args.ksplit; s0 += 8) {
+            float pp[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int q8 = 0; q8 < 8; ++q8)
+                pp[u][q8] = (in[u] && s0 + q8 < args.ksplit) ? __ldcg(args.zpart + (size_t)(s0 + q8) * plane + o[u]) : 0.0f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int q8 = 0; q8 < 8; ++q8)
+                if (s0 + q8 < args.ksplit) v[u] += pp[u][q8];
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (in[u]) args.z[o[u]] = args.bias ? v[u] + __ldg(args.bias + (int)(o[u] % args.E)) : v[u];
         }
       }
       __threadfence();
@@ -296,12 +322,18 @@ __global__ void __launch_bounds__(320, 1)
       if (!last_flag[1]) continue;
       __threadfence();                                 // every logit of the token tile is visible
       const int ew = warp - 2;
-      if (ew < args.topk_warps) {
+      if (args.E <= 32 * kTopkKeysPerLane) {
+        for (int n = ew; n < n_valid; n += 8) {
+          const size_t t_ = (size_t)(row0 + n);
+          topk_sigmoid_row_regs(args.z + t_ * args.E, args.sel_bias, args.E, args.k, args.idx + t_ * args.k,
+                                args.w + t_ * args.k, lane);
+        }
+      } else if (ew < args.topk_warps) {
         float* row = topk_rows + (size_t)ew * args.E;
         for (int n = ew; n < n_valid; n += args.topk_warps) {
           const size_t t_ = (size_t)(row0 + n);
-          topk_sigmoid_row(args.z + t_ * args.E, args.sel_bias, args.E, args.k, row, args.idx + t_ * args.k,
-                           args.w + t_ * args.k, lane);
+          topk_sigmoid_row_smem(args.z + t_ * args.E, args.sel_bias, args.E, args.k, row, args.idx + t_ * args.k,
+                                args.w + t_ * args.k, lane);
         }
       }
     }

@@ -276,13 +276,14 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  *   this many K tiles ahead of the shared-memory loads (0..64, 0 = off).
  * MOE_OPT_PREFETCH_B: accepted and ignored (reserved).
  * MOE_OPT_TILE_N: token rows per routed grouped-GEMM tile.  0 (default) picks per call:
- *   128 rows when T*k <= 96*E (most experts within one tile), with the token rows on the
- *   MMA's M side and 256 weight rows on its N side; else 176 rows with the weights on M
- *   and the tokens on N.  32 selects a third configuration (weights on M, 32 token rows,
- *   5-stage pipeline).  32, 128 or 176 forces one configuration; any other value is
- *   MOE_ERR_INVALID_ARG.  The dense shared-expert GEMMs use 32-row tiles when T*k <= 8*E
- *   and 176 otherwise.  Results agree within fp32 accumulation (the K loop runs in the same
- *   order in all three).
+ *   32 rows (5-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure
+ *   weight stream, else 176 rows (4 stages); both put 256 weight rows on the MMA's M side
+ *   and the token rows on its N side.  128 selects the other orientation: token rows on M
+ *   (up to 128 per tile) and 256 weight rows on N.  32, 128 or 176 forces one
+ *   configuration; any other value is MOE_ERR_INVALID_ARG.  The dense shared-expert GEMMs
+ *   use 32-row tiles when T*k <= 8*E and 176 otherwise.  The K loop runs in the same order
+ *   in all three, and the tensor core accumulates a row the same way in either
+ *   orientation: results are identical.
  * MOE_OPT_ROUTER_SPLIT (read only): the number of K splits the last moe_route used for
  *   the router GEMM (1 = none).  With few tokens the router splits d over up to one
  *   CTA per SM; the CTA that finishes a tile's last split adds the fp32 partials in split

@@ -12,7 +12,8 @@
  *     value list (ties to the even code), saturating at the largest entry (R1), with the
  *     sign bit of v kept, also for a value that rounds to zero (R2).
  * The positive value lists come from the caller (oracle/mx.py builds them from the formats'
- * sign/exponent/mantissa definitions), so the two restatements share one table.
+ * sign/exponent/mantissa definitions), so the two restatements share one table.  The
+ * decoder (mx_dequantize_f64) restates oracle/mx.py's dequantize_mx the same way.
  */
 #include <math.h>
 #include <stdint.h>
@@ -67,6 +68,22 @@ void mx_quantize_f32(const float* v, long rows, long K, const double* pos, int n
         const int idx = nearest_even(pos, n, a);
         codes[r * K + b * 32 + i] = (uint8_t)(idx | (signbit(q) ? sign_bit : 0));
       }
+    }
+  }
+}
+
+/* Exact fp64 values of MX data: table[code & code_mask] * 2^(scale - 127) per block of 32
+ * (a scale byte of 0xFF is NaN).  codes: uint8 [rows][K]; scales: uint8 [rows][K / 32];
+ * table: the format's value of every code (16 or 256 entries, from oracle/mx.py). */
+void mx_dequantize_f64(const uint8_t* codes, const uint8_t* scales, long rows, long K, const double* table,
+                       int code_mask, double* out) {
+  for (long r = 0; r < rows; ++r) {
+    for (long b = 0; b < K / 32; ++b) {
+      const int sb = scales[r * (K / 32) + b];
+      const double sc = sb == 255 ? NAN : ldexp(1.0, sb - 127);
+      const uint8_t* c = codes + r * K + b * 32;
+      double* o = out + r * K + b * 32;
+      for (int i = 0; i < 32; ++i) o[i] = table[c[i] & code_mask] * sc;
     }
   }
 }

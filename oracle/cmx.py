@@ -1,8 +1,8 @@
-"""ctypes wrapper of oracle/cmx.c: the MX block quantiser of oracle/mx.py restated in C.
-TEST INFRASTRUCTURE ONLY.
+"""ctypes wrapper of oracle/cmx.c: the MX block quantiser and decoder of oracle/mx.py
+restated in C.  TEST INFRASTRUCTURE ONLY.
 
-Same rule, same value tables (taken from oracle.mx), same results: pinned bit-exact
-against ``oracle.mx.quantize_mx`` by ``tests/test_oracle_mx.py``.  It exists so that the
+Same rules, same value tables (taken from oracle.mx), same results: pinned bit-exact
+against ``oracle.mx.quantize_mx`` / ``dequantize_mx`` by ``tests/test_oracle_mx.py``.  It exists so that the
 parity tests at the Kimi-K3 shapes can quantise many experts' weights quickly.  ``build()``
 compiles it with gcc into ``oracle/_cmx.so`` (it is built on first use when missing).
 """
@@ -37,6 +37,10 @@ def _load():
         f.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                       ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
         f.restype = None
+        g = L.mx_dequantize_f64
+        g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_void_p, ctypes.c_int,
+                      ctypes.c_void_p]
+        g.restype = None
         _lib = L
     return _lib
 
@@ -59,3 +63,17 @@ def quantize_mx_f32(values, fmt):
     _load().mx_quantize_f32(v.ctypes.data, rows, K, pos.ctypes.data, len(pos), emax, sign_bit,
                             codes.ctypes.data, scales.ctypes.data)
     return codes, scales
+
+
+def dequantize_mx_f64(codes, scales, fmt):
+    """dequantize_mx: exact fp64 values of MX codes [..., K] with scale bytes [..., K/32],
+    equal to oracle.mx.dequantize_mx(codes, scales, fmt)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    sc = np.ascontiguousarray(scales, dtype=np.uint8)
+    K = c.shape[-1]
+    table, mask = (mx.E2M1_TABLE, 15) if fmt == "e2m1" else (mx.E4M3_TABLE, 255)
+    table = np.ascontiguousarray(table, dtype=np.float64)
+    out = np.empty(c.shape, dtype=np.float64)
+    _load().mx_dequantize_f64(c.ctypes.data, sc.ctypes.data, c.size // K, K, table.ctypes.data, mask,
+                              out.ctypes.data)
+    return out

@@ -18,6 +18,7 @@ Nothing here reads kernel output: the token rows, routing and weights are the or
 """
 import os
 from collections import deque
+from multiprocessing import shared_memory
 
 import numpy as np
 import torch
@@ -48,14 +49,38 @@ def quantize_expert_fast(W_gate, W_up, W_down):
             "down": cmx.quantize_mx_f32(W_down, "e2m1")}
 
 
-def expert_job(w_gate, w_up, w_down, blocks, want_stage, act):
+def decode_expert_fast(q):
+    """oracle.layer.decode_expert with the C restatement of the MX decoder (pinned
+    bit-exact against oracle.mx.dequantize_mx)."""
+    return tuple(cmx.dequantize_mx_f64(*q[name], "e2m1") for name in ("gate", "up", "down"))
+
+
+# worker side: shared-memory blocks attached once per process, by name
+_attached = {}
+
+
+def _masters(name, shapes):
+    if name not in _attached:
+        _attached[name] = shared_memory.SharedMemory(name=name)
+    buf = _attached[name].buf
+    out, off = [], 0
+    for shp in shapes:
+        n = int(np.prod(shp))
+        out.append(np.ndarray(shp, dtype=np.float32, buffer=buf, offset=off))
+        off += 4 * n
+    return out
+
+
+def expert_job(shm_name, shapes, blocks, want_stage, act):
     """Worker: one expert's oracle outputs for several blocks of decoded token rows.
 
-    w_*: fp32 masters (torch CPU tensors in shared memory); blocks: list of fp64 [R, d]
-    arrays.  Returns, per block, (o,) or, with want_stage, (o, a, hq, hs)."""
+    shm_name/shapes: the fp32 masters (gate, up, down) in a shared-memory block; blocks:
+    list of fp64 [R, d] arrays.  Returns, per block, (o,) or, with want_stage,
+    (o, a, hq, hs)."""
     torch.set_num_threads(1)
-    q = quantize_expert_fast(w_gate.numpy(), w_up.numpy(), w_down.numpy())
-    Wg, Wu, Wd = layer.decode_expert(q)
+    w_gate, w_up, w_down = _masters(shm_name, shapes)
+    q = quantize_expert_fast(w_gate, w_up, w_down)
+    Wg, Wu, Wd = decode_expert_fast(q)
     out = []
     for X in blocks:
         o, a, hq, hs = layer.expert_forward(X, Wg, Wu, Wd, act)
@@ -67,24 +92,40 @@ def run_experts(wl, jobs, stage_experts=(), act="silu", device=None):
     """jobs: {expert: [fp64 [R, d] token-row block, ...]} -> {expert: [result per block]}.
 
     Results are expert_job's tuples; experts in `stage_experts` also return the GLU values
-    and their MXFP8 codes and scales."""
+    and their MXFP8 codes and scales.  The parent draws each expert's masters straight into
+    one of 2 x pool-size shared-memory blocks, reused round robin (a block is rewritten only
+    after the job that read it has returned)."""
     import torch.multiprocessing as tmp
     device = wl.device if device is None else device
     n = pool_size()
     ctx = tmp.get_context("spawn")
+    de = wl.d_expert
+    shapes = ((wl.I, de), (wl.I, de), (de, wl.I))
+    nbytes = 4 * sum(a * b for a, b in shapes)
+    blocks_shm = [shared_memory.SharedMemory(create=True, size=nbytes) for _ in range(2 * n)]
     results = {}
-    with ctx.Pool(n) as pool:
-        inflight = deque()
-        for e in sorted(jobs):
-            while len(inflight) >= 2 * n:            # bound the masters held in shared memory
+    try:
+        with ctx.Pool(n) as pool:
+            inflight = deque()
+            for i, e in enumerate(sorted(jobs)):
+                while len(inflight) >= 2 * n:            # frees the block this job reuses
+                    e0, r0 = inflight.popleft()
+                    results[e0] = r0.get()
+                blk = blocks_shm[i % (2 * n)]
+                off = 0
+                for t, shp in zip(synth.draw_expert(wl, e, device=device), shapes):
+                    cnt = shp[0] * shp[1]
+                    dst = torch.from_numpy(np.ndarray(shp, dtype=np.float32, buffer=blk.buf, offset=off))
+                    dst.copy_(t)
+                    off += 4 * cnt
+                inflight.append((e, pool.apply_async(expert_job, (blk.name, shapes, jobs[e], e in stage_experts, act))))
+            while inflight:
                 e0, r0 = inflight.popleft()
                 results[e0] = r0.get()
-            ms = [t.cpu().share_memory_() for t in synth.draw_expert(wl, e, device=device)]
-            inflight.append((e, pool.apply_async(expert_job, (*ms, jobs[e], e in stage_experts, act))))
-            del ms
-        while inflight:
-            e0, r0 = inflight.popleft()
-            results[e0] = r0.get()
+    finally:
+        for b in blocks_shm:
+            b.close()
+            b.unlink()
     return results
 
 

@@ -221,8 +221,8 @@ def test_layer_tile_configs_agree():
     """The three routed-GEMM tile configurations (32 and 176 token rows with the weights on
     the MMA's M side, 128 with the tokens on M) on one input whose hot experts span several
     tiles in each (400 rows: 13 tiles of <= 32 rows, 4 of <= 128, 3 of <= 176): each matches
-    the oracle.  The two weights-on-M configurations give the same bytes (the K loop runs in
-    the same order); the tokens-on-M one agrees with them within fp32 accumulation."""
+    the oracle, and all three give the same bytes: the K loop runs in the same order, and
+    the tensor core accumulates an output the same way in either orientation."""
     wl = synth.custom(seed=11, T=400, d=256, E=16, k=4, I=128, I_shared=128)
     bias = torch.zeros(16)
     bias[[1, 5, 6, 14]] = 40.0
@@ -234,10 +234,7 @@ def test_layer_tile_configs_agree():
         assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_TILE_N) == bn
         idx, w = case.plan.route(case.x, case.W_r, case.bias)
         outs.append(case.plan.forward(case.x, idx, w, case.experts, case.shared).cpu())
-    assert torch.equal(outs[0], outs[2])
-    diff = (outs[1].float() - outs[2].float()).abs()
-    print("tokens-on-M vs weights-on-M: max |diff|", float(diff.max()), "elements differing", int((diff > 0).sum()))
-    assert float(diff.max()) <= 2.0 ** -6 * float(outs[2].float().abs().max())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 0)
     with pytest.raises(api.MoeError):
         api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 64)
@@ -440,3 +437,34 @@ def test_route_and_forward_replay_from_a_cuda_graph():
     torch.cuda.synchronize()
     assert torch.equal(y, y_eager)
     assert case.plan.check()[0] == 0
+
+
+@pytest.mark.parametrize("E,k,select_only", [(96, 8, False), (1100, 16, False), (64, 4, True)])
+def test_route_exact_ties_lower_index_wins(E, k, select_only):
+    """Exact ties in the selection key: duplicated router columns give equal logits, an
+    all-zero token gives every expert the logit +0 (and -0 where the bias is -0), and in the
+    select-only mode equal keys come from different (z, b) pairs.  The selection on the
+    GPU's own logits must equal the oracle's (descending key, lower index first), also with
+    more experts than the register form holds (E = 1100 takes the shared-memory form)."""
+    T, d = 40, 128
+    g = torch.Generator().manual_seed(E + k)
+    x = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    x[3] = 0.0
+    W_r = torch.randn((d, E), generator=g) * 0.02
+    W_r[:, 1::3] = W_r[:, 0::3][:, :W_r[:, 1::3].shape[1]]       # every third pair of experts ties
+    b = torch.zeros(E)
+    b[::5] = -0.0
+    if select_only:
+        b = torch.randint(-2, 3, (E,), generator=g).float() * 0.5
+    plan = api.Plan(T, d, E, k, 128, bias_mode=api.MOE_BIAS_SELECT_ONLY if select_only else api.MOE_BIAS_LOGIT)
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    idx, w = plan.route(x.cuda(), W_r.cuda(), b.cuda(), logits=logits)
+    z = logits.cpu().numpy()
+    if select_only:
+        idx_g, w_g, _ = router.route(z, k, select_bias=b.numpy())
+    else:
+        idx_g, w_g, _ = router.route(z.astype(np.float64), k)
+    assert np.array_equal(idx.cpu().numpy(), idx_g)
+    assert np.allclose(w.cpu().numpy(), w_g, rtol=2e-6, atol=1e-7)
+    if not select_only:
+        assert list(idx[3].cpu().numpy()) == list(range(k))     # all logits tie at zero

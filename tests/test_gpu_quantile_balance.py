@@ -88,7 +88,9 @@ def test_quantile_balance_calls_the_rule_with_this_steps_quantiles():
         # the test's own rule (the pages publish none): move each expert's bias half way
         # towards putting its (1 - k/E)-quantile margin at zero, on the call's stream
         seen.update(q=q_ptr, n=n_levels, E=n_experts, b=b_ptr, nxt=next_ptr, user=user)
-        with torch.cuda.stream(torch.cuda.ExternalStream(stream_ptr)):
+        # a NULL stream is the legacy default stream, which torch calls its default stream
+        st = torch.cuda.ExternalStream(stream_ptr) if stream_ptr else torch.cuda.default_stream()
+        with torch.cuda.stream(st):
             nxt.copy_(bias - 0.5 * qview[0])
 
     cb = api.BIAS_RULE(rule)

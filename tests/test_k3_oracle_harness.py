@@ -17,6 +17,14 @@ def test_fast_expert_quantiser_matches_the_oracle():
         assert np.array_equal(a[name][0], b[name][0]) and np.array_equal(a[name][1], b[name][1])
 
 
+def test_fast_expert_decoder_matches_the_oracle():
+    g = np.random.default_rng(4)
+    ms = [(g.standard_normal(s) * 0.02).astype(np.float32) for s in ((64, 256), (64, 256), (256, 64))]
+    q = layer.quantize_expert(*ms)
+    for a, b in zip(k3_oracle.decode_expert_fast(q), layer.decode_expert(q)):
+        assert np.array_equal(a, b)
+
+
 def test_pool_layer_outputs_match_single_process_oracle():
     wl = synth.custom(seed=8, T=40, d=256, E=8, k=3, I=128, I_shared=128)
     x = synth.draw_x(wl).float().numpy().astype(np.float64)

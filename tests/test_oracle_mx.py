@@ -217,3 +217,19 @@ def test_c_quantiser_round_trips_every_code():
                 assert scales[0, 0] == s + 127       # amax = largest value x 2^s: exponent s
                 dec = mx.dequantize_mx(codes, scales, fmt)
                 assert dec[0, 1] == blk[1] and dec[0, 2] == blk[2], (fmt, s, c)
+
+
+def test_c_decoder_matches_the_numpy_definition():
+    """oracle/cmx.c's decoder gives dequantize_mx's values: every code with a spread of
+    scale bytes, the NaN scale (0xFF) and the E4M3 NaN codes included."""
+    from oracle import cmx
+    g = np.random.default_rng(13)
+    for fmt, ncodes in (("e2m1", 16), ("e4m3", 256)):
+        codes = g.integers(0, ncodes, size=(64, 256)).astype(np.uint8)
+        codes[0, :ncodes] = np.arange(ncodes)
+        scales = g.integers(0, 256, size=(64, 8)).astype(np.uint8)
+        scales[1] = 255
+        scales[2] = [0, 1, 126, 127, 128, 253, 254, 255]
+        a = cmx.dequantize_mx_f64(codes, scales, fmt)
+        b = mx.dequantize_mx(codes, scales, fmt)
+        assert np.array_equal(a, b, equal_nan=True), fmt
