@@ -52,8 +52,8 @@ SIGNATURES = {
 
 STAGES = ["router_split", "router_gemm", "topk", "permute", "quant_scatter", "gate_up_glu",
           "down", "shared_gate_up", "shared_down", "combine", "latent_in", "latent_out"]
-# kernel launches per recorded stage instance (the router kernel also sums its K-split
-# partials and selects the top-k, so "topk" records nothing)
+# kernel launches per recorded stage instance ("topk" is the selection kernel, which also
+# sums the router GEMM's K-split partials)
 STAGE_KERNELS = {"permute": 3, "quant_scatter": 2, "latent_in": 2, "latent_out": 2}
 
 

@@ -38,7 +38,7 @@ constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
 constexpr int kRouterStages = 3;
 constexpr int kRouterMaxCtas = 256;   // bound on split router tiles (sizes the partials)
-constexpr int kMaxDynSmem = 232448;   // opt-in dynamic shared memory per block (227 KB)
+constexpr int kMaxExperts = 4096;
 constexpr int kSplitMaxCtas = 256;    // bound on split-K dense GEMM tiles (sizes their partials)
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -153,7 +153,7 @@ struct moe_plan_s {
   size_t ws_bytes = 0;
   // workspace carve (byte offsets)
   size_t o_status, o_chunk, o_counts, o_offsets, o_tiles, o_perm, o_inv, o_logits, o_zpart,
-      o_planes, o_rcnt, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_spart, o_theta, o_qbuf, o_xl, o_xn, o_yl,
+      o_planes, o_xq, o_xs_tok, o_xs, o_hq, o_hs, o_O, o_hsh, o_ys, o_spart, o_theta, o_qbuf, o_xl, o_xn, o_yl,
       o_yr, total;
   int dl = 0;              // latent option: expert width (0 = off)
   float eps_lat = 1e-5f;
@@ -180,11 +180,6 @@ static void carve(moe_plan_s* p) {
   p->zpart_floats = std::max((size_t)kRouterMaxCtas * kRouterBN * 128, (size_t)3 * p->T_max * p->E);
   p->o_zpart = take(p->zpart_floats * 4);
   p->o_planes = take((size_t)p->E * 3 * p->d * 2);
-  // fused router selection counters: [token tiles][expert tiles] splits done + [token tiles]
-  {
-    const size_t n_tt = (size_t)(std::max(p->T_max, 1) + kRouterBN - 1) / kRouterBN;
-    p->o_rcnt = take((n_tt * ((p->E + 127) / 128) + n_tt) * sizeof(int));
-  }
   p->o_xq = take(A * p->d);
   // token-side scale blocks, tile-major: at most A / bn + E group-tiles
   const size_t max_tiles = A / kBNMin + p->E + 1;
@@ -319,7 +314,7 @@ moe_status_t moe_plan_create(int T_max, int d, int E, int k, int I, int I_shared
       (bias_mode != MOE_BIAS_LOGIT && bias_mode != MOE_BIAS_SELECT_ONLY) || (flags & ~MOE_FLAG_STATIC_ROUTER))
     return MOE_ERR_INVALID_ARG;
   if (T_max < 0 || d <= 0 || E <= 0 || k <= 0 || I <= 0 || I_shared < 0) return MOE_ERR_INVALID_ARG;
-  if (d % 128 || I % 128 || I_shared % 128 || k > E || k > 32 || E > 4096)
+  if (d % 128 || I % 128 || I_shared % 128 || k > E || k > 32 || E > kMaxExperts)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((long long)T_max * k > (1ll << 30)) return MOE_ERR_UNSUPPORTED_SHAPE;
   moe_plan_s* p = new moe_plan_s();
@@ -442,16 +437,9 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   // MOE_BIAS_SELECT_ONLY: z stays unbiased; the bias only enters the top-k key
   const bool select_only = p->bias_mode == MOE_BIAS_SELECT_ONLY;
   ra.bias = select_only ? nullptr : bias;
-  ra.sel_bias = select_only ? bias : nullptr;
   ra.z = z;
   ra.zpart = p->at<float>(p->o_zpart);
   ra.status = p->at<unsigned int>(p->o_status);
-  ra.k = p->k;
-  ra.idx = idx;
-  ra.w = w;
-  const int n_tt = (T + kRouterBN - 1) / kRouterBN;
-  ra.cnt_split = p->at<int>(p->o_rcnt);
-  ra.cnt_tile = ra.cnt_split + (size_t)n_tt * ra.m_tiles;
   {
     // Split K (i) when the expert x token tiles would fill less than half the SMs, so that
     // the plane reads (3 x E x d bf16) spread over the whole GPU, and (ii) otherwise by up
@@ -480,20 +468,37 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     p->last_ksplit = ra.ksplit;
     using RC = RouterCfg<kRouterBN, kRouterStages>;
     auto kern = router_kernel<kRouterBN, kRouterStages>;
-    // the fused selection holds the keys in registers up to E = 1024; beyond, one E-float
-    // shared-memory row per selecting warp after the pipeline
-    ra.topk_warps = E <= 32 * kTopkKeysPerLane ? 0 : std::min(8, (kMaxDynSmem - RC::SMEM_BYTES) / (E * 4));
-    if (E > 32 * kTopkKeysPerLane && ra.topk_warps < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
-    const int smem = RC::SMEM_BYTES + ra.topk_warps * E * 4;
     static std::atomic<uint64_t> router_done{0};
-    if (ensure_smem_attr(kern, kMaxDynSmem, router_done) != cudaSuccess) return MOE_ERR_CUDA;
+    if (ensure_smem_attr(kern, RC::SMEM_BYTES, router_done) != cudaSuccess) return MOE_ERR_CUDA;
     const int tiles = base_tiles * ra.ksplit;
     p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
-    // the selection counters start from zero every call
-    if (cudaMemsetAsync(ra.cnt_split, 0, ((size_t)n_tt * ra.m_tiles + n_tt) * sizeof(int), s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    kern<<<std::min(tiles, p->num_sms), 320, smem, s>>>(ra, tA, tB);
+    kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    p->prof.end(s);
+  }
+  {
+    // selection (and, after a K split, the sum of the partials): 8 tokens per CTA when
+    // there are enough to fill the GPU that way, else one; their keys in shared memory
+    const int tpc = T >= 8 * p->num_sms ? 8 : 1;
+    const int grid = std::min((T + tpc - 1) / tpc, 32 * p->num_sms);
+    const float* sel = select_only ? bias : nullptr;
+    const float* lbias = select_only ? nullptr : bias;
+    const long long plane = (long long)T * E;
+    const int k = p->k;
+    const int smem = tpc * E * 4;   // <= 8 * 4096 * 4 = 128 KB
+    cudaError_t err = cudaSuccess;
+    auto launch = [&](auto kern, std::atomic<uint64_t>& done) {
+      err = ensure_smem_attr(kern, 8 * kMaxExperts * 4, done);
+      if (err == cudaSuccess) kern<<<grid, 256, smem, s>>>(ra.zpart, ra.ksplit, plane, lbias, sel, z, T, E, k, tpc, idx, w);
+    };
+    static std::atomic<uint64_t> sel_done[5];
+    p->prof.begin(MOE_STAGE_TOPK, s);
+    if (E <= 256)       launch(route_select_kernel<1>, sel_done[0]);
+    else if (E <= 512)  launch(route_select_kernel<2>, sel_done[1]);
+    else if (E <= 1024) launch(route_select_kernel<4>, sel_done[2]);
+    else if (E <= 2048) launch(route_select_kernel<8>, sel_done[3]);
+    else                launch(route_select_kernel<16>, sel_done[4]);
+    if (err != cudaSuccess || cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
   p->last_T = T;
@@ -1023,7 +1028,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* idx, int T, int E, in
                                             int32_t* offsets, int32_t* perm_tok, int32_t* inv,
                                             void* stream) {
   if (T < 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
-  if (k > E || k > 32 || E > 4096) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (k > E || k > 32 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!counts || !offsets || (T > 0 && (!idx || !perm_tok || !inv))) return MOE_ERR_INVALID_ARG;
   const int nch = (T + kPermThreads - 1) / kPermThreads;
   const size_t o_chunk = 256, o_tiles = o_chunk + up((size_t)nch * E * 4, 256);

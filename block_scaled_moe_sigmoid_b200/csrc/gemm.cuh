@@ -30,10 +30,11 @@
 // Orientation WN (KIND_MX, a few tokens per expert): the token rows are the MMA's M side
 // (128 lanes, of which the tile's rows are the first n) and all 256 weight rows of the tile
 // are its N side, so each K block is one M=128 x N=256 instruction instead of two M=128 x
-// N=n ones.  Issued back to back from one thread, a block-scaled M=128 tcgen05.mma takes
-// the same time for every N from 16 to 256 (measured: ~135 cycles at 1965 MHz, about the
-// N=256 execution time), so with few tokens this halves the time per weight byte, and the
-// weight stream is what the kernel is there for.
+// N=n ones.  Issued back to back from one thread, a block-scaled M=128 x N x K=32
+// tcgen05.mma takes max(~51, N/2) cycles (the N/2 is the FP8 rate; ~51 is the issue floor
+// of one thread), so with few tokens one N=256 instruction (128 cycles) replaces two
+// floor-bound ones (~102).  Measured, it is slower all the same (fewer pipeline stages fit);
+// it stays selectable.
 // The accumulator is then tokens x (gate | up) or tokens x output channels; the epilogue
 // reads a token row per thread.  Shared memory, producers and scale copies are as above
 // (the weight scales become the B side's, the token scales the A side's).

@@ -315,89 +315,176 @@ __device__ __forceinline__ float f32_from_order_key(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-// Selection for one token, by one warp: key = z (+ select_bias in the select-only mode,
-// fp32); the k largest keys in descending order, the lower expert index first among equal
-// keys; then w_j = s_j / sum of the selected s, s = sigmoid(z).  z is read through L2
-// (__ldcg): it may have been written by other CTAs of the same kernel.
-//
-// Fast form (E <= 32 * KPL): each lane keeps the keys of experts lane, lane + 32, ... in
-// registers.  A round takes the lane's first largest key, then the warp's largest as a
-// redux.sync max of an order-preserving uint32 map, then the lowest index among the lanes
-// holding it as a redux.sync min; the owning lane marks that key taken.
-constexpr int kTopkKeysPerLane = 32;
-__device__ __forceinline__ void topk_sigmoid_row_regs(const float* __restrict__ z_row,
-                                                      const float* __restrict__ select_bias, int E, int k,
-                                                      int* __restrict__ idx_out, float* __restrict__ w_out,
-                                                      int lane) {
-  float v[kTopkKeysPerLane];
+// Top-k selection: the k largest keys in descending order, the lower expert index first
+// among equal keys, by warp rounds over per-lane candidate lists.  Each lane holds C (order key, expert index) pairs sorted by key
+// descending, lower index first among equal keys; a round takes the warp's best head (a
+// redux.sync max of the keys, then a redux.sync min of the indices holding it) and the
+// owning lane drops its head.  An empty slot is (0, 0x7fffffff): below every finite key's
+// order key, and never chosen while k real candidates remain.
+constexpr uint32_t kEmptyIdx = 0x7fffffffu;
+
+template <int C>
+__device__ __forceinline__ void lane_sort_desc(uint32_t (&key)[C], uint32_t (&idx)[C]) {
+  // odd-even transposition: C passes sort C entries
 #pragma unroll
-  for (int j = 0; j < kTopkKeysPerLane; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = e < E ? (select_bias ? __ldcg(z_row + e) + __ldg(select_bias + e) : __ldcg(z_row + e)) : -INFINITY;
-  }
-  float ssum = 0.0f, my_s = 0.0f;
-  int my_i = -1;
-  uint32_t taken = 0;   // bit j: key j of this lane already selected (v itself is never rewritten)
-  for (int r = 0; r < k; ++r) {
-    float bv = (taken & 1u) ? -INFINITY : v[0];
-    int bj = 0;
+  for (int r = 0; r < C; ++r)
 #pragma unroll
-    for (int j = 1; j < kTopkKeysPerLane; ++j) {
-      const float vj = ((taken >> j) & 1u) ? -INFINITY : v[j];
-      if (vj > bv) { bv = vj; bj = j; }        // ascending index: the first max is kept
+    for (int i = r & 1; i + 1 < C; i += 2) {
+      const bool sw = key[i] < key[i + 1] || (key[i] == key[i + 1] && idx[i] > idx[i + 1]);
+      const uint32_t k0 = sw ? key[i + 1] : key[i], k1 = sw ? key[i] : key[i + 1];
+      const uint32_t i0 = sw ? idx[i + 1] : idx[i], i1 = sw ? idx[i] : idx[i + 1];
+      key[i] = k0; key[i + 1] = k1;
+      idx[i] = i0; idx[i + 1] = i1;
     }
-    const uint32_t bu = f32_order_key(bv + 0.0f);   // -0 -> +0: equal keys compare equal
-    const uint32_t mu = __reduce_max_sync(0xffffffffu, bu);
-    const uint32_t cand = bu == mu ? (uint32_t)(lane + 32 * bj) : 0xffffffffu;
-    const int bi = (int)__reduce_min_sync(0xffffffffu, cand);
-    const float zsel = select_bias ? __ldcg(z_row + bi) : f32_from_order_key(mu);
-    const float s = 1.0f / (1.0f + expf(-zsel));
-    ssum += s;
-    if (lane == r) { my_s = s; my_i = bi; }
-    if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
-  }
-  if (lane < k) {
-    idx_out[lane] = my_i;
-    w_out[lane] = my_s / ssum;
-  }
-  __syncwarp();
 }
 
-// General form (any E): the keys in the warp's shared-memory row of E floats; k rounds of a
-// warp arg-max (shuffles, lower index on equal keys).
-__device__ __forceinline__ void topk_sigmoid_row_smem(const float* __restrict__ z_row, const float* __restrict__ select_bias,
-                                                      int E, int k, float* row, int* __restrict__ idx_out,
-                                                      float* __restrict__ w_out, int lane) {
-  for (int e = lane; e < E; e += 32)
-    row[e] = select_bias ? __ldcg(z_row + e) + __ldg(select_bias + e) : __ldcg(z_row + e);
-  __syncwarp();
-  float ssum = 0.0f, my_s = 0.0f;
-  int my_i = -1;
+// k rounds over sorted per-lane lists; lane r (< k) receives the r-th selection.
+template <int C>
+__device__ __forceinline__ void warp_select_lists(uint32_t (&key)[C], uint32_t (&idx)[C], int k, int lane,
+                                                  uint32_t& my_key, uint32_t& my_idx) {
+  my_key = 0;
+  my_idx = kEmptyIdx;
   for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) {
-      const float v = row[e];
-      if (v > bv) { bv = v; bi = e; }  // ascending e: first max kept on ties
-    }
+    const uint32_t mu = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t bi = __reduce_min_sync(0xffffffffu, key[0] == mu ? idx[0] : 0xffffffffu);
+    if (lane == r) { my_key = mu; my_idx = bi; }
+    if (key[0] == mu && idx[0] == bi) {   // the winner drops its head
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      for (int i = 0; i + 1 < C; ++i) { key[i] = key[i + 1]; idx[i] = idx[i + 1]; }
+      key[C - 1] = 0;
+      idx[C - 1] = kEmptyIdx;
     }
-    const float zsel = select_bias ? __ldcg(z_row + bi) : bv;
-    const float s = 1.0f / (1.0f + expf(-zsel));
-    ssum += s;
-    if (lane == r) { my_s = s; my_i = bi; }
-    if (lane == 0) row[bi] = -INFINITY;
-    __syncwarp();
   }
-  if (lane < k) {
-    idx_out[lane] = my_i;
-    w_out[lane] = my_s / ssum;
+}
+
+// Route selection, one launch after the router GEMM.  A CTA of 8 warps takes `tpc` tokens
+// (1 or 8) at a time.
+//   Stage 1: warp w owns the expert slice [w * 32C, (w + 1) * 32C), C experts per lane; it
+//   forms z (the split partials summed in split order, plus the logit bias, stored; or z
+//   as the GEMM stored it) and the selection key (z, or z + b in the select-only mode,
+//   fp32) as an order-preserving uint32 in shared memory.
+//   Stage 2: warp i selects token i's top k from its E keys.  theta = the k-th largest of
+//   the 32 lanes' maxima: k lanes hold a key >= theta, so the k-th largest key is >= theta,
+//   and every key of the top k (ties at the k-th included) is >= theta.  Those candidates,
+//   about 20 of 896 for spread keys, go into per-lane lists of 4 and k warp rounds pick
+//   them in order (key descending, lower index first).  When some lane holds more than 4
+//   (heavy ties), the rounds scan the keys in shared memory instead.
+//   Then w_j = s_j / sum of the selected s, s = sigmoid(z), the sum in selection order.
+// z is not __restrict__: stage 2 reads back what stage 1 stored.
+template <int C>
+__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ zpart, int ksplit,
+                                                           long long plane, const float* __restrict__ bias,
+                                                           const float* __restrict__ select_bias, float* z, int T,
+                                                           int E, int k, int tpc, int* __restrict__ idx_out,
+                                                           float* __restrict__ w_out) {
+  extern __shared__ uint32_t sel_keys[];   // [tpc][E] order keys
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t0 = blockIdx.x * tpc; t0 < T; t0 += gridDim.x * tpc) {
+    // ---- stage 1
+    for (int i = 0; i < tpc && t0 + i < T; ++i) {
+      const size_t row = (size_t)(t0 + i) * E;
+      float v[C];
+#pragma unroll
+      for (int c = 0; c < C; ++c) v[c] = 0.0f;
+      if (ksplit > 1) {
+        constexpr int S = C >= 8 ? 2 : 8;   // partials in flight per expert
+        for (int s0 = 0; s0 < ksplit; s0 += S) {
+          float pp[C][S];
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const int e = warp * 32 * C + lane + 32 * c;
+#pragma unroll
+            for (int q = 0; q < S; ++q)
+              pp[c][q] = (e < E && s0 + q < ksplit) ? __ldcg(zpart + (size_t)(s0 + q) * plane + row + e) : 0.0f;
+          }
+#pragma unroll
+          for (int c = 0; c < C; ++c)
+#pragma unroll
+            for (int q = 0; q < S; ++q)
+              if (s0 + q < ksplit) v[c] = (s0 + q == 0) ? pp[c][q] : v[c] + pp[c][q];
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const int e = warp * 32 * C + lane + 32 * c;
+        if (e < E) {
+          float zv;
+          if (ksplit > 1) {
+            zv = bias ? v[c] + __ldg(bias + e) : v[c];
+            z[row + e] = zv;
+          } else {
+            zv = z[row + e];
+          }
+          const float kv = select_bias ? zv + __ldg(select_bias + e) : zv;
+          sel_keys[(size_t)i * E + e] = f32_order_key(kv + 0.0f);   // -0 -> +0: equal keys compare equal
+        }
+      }
+    }
+    __syncthreads();
+    // ---- stage 2
+    if (warp < tpc && t0 + warp < T) {
+      const int t = t0 + warp;
+      uint32_t* kr = sel_keys + (size_t)warp * E;
+      uint32_t lmax = 0;
+      for (int e = lane; e < E; e += 32) lmax = max(lmax, kr[e]);
+      // theta: k rounds of the warp maximum over the lane maxima, one holder removed a round
+      uint32_t theta = 0, mk = lmax;
+      for (int r = 0; r < k; ++r) {
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, mk);
+        theta = mx;
+        const uint32_t bl = __reduce_min_sync(0xffffffffu, mk == mx ? (uint32_t)lane : 32u);
+        if ((uint32_t)lane == bl) mk = 0;
+      }
+      uint32_t key[4], id[4];
+      int cnt = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { key[j] = 0; id[j] = kEmptyIdx; }
+      for (int e = lane; e < E; e += 32) {
+        const uint32_t kv = kr[e];
+        if (kv >= theta) {
+          // append at slot cnt (predicated writes: no dynamic register index)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (j == cnt) { key[j] = kv; id[j] = (uint32_t)e; }
+          ++cnt;
+        }
+      }
+      uint32_t sk, si;
+      if (__any_sync(0xffffffffu, cnt > 4)) {
+        // heavy ties: k rounds over all keys; a taken key becomes 0 (below every real key)
+        sk = 0;
+        si = kEmptyIdx;
+        for (int r = 0; r < k; ++r) {
+          uint32_t bv = 0, bi = kEmptyIdx;
+          for (int e = lane; e < E; e += 32) {
+            const uint32_t kv = kr[e];
+            if (kv > bv) { bv = kv; bi = (uint32_t)e; }   // ascending e: the lower index kept
+          }
+          const uint32_t mu = __reduce_max_sync(0xffffffffu, bv);
+          const uint32_t wi = __reduce_min_sync(0xffffffffu, bv == mu ? bi : 0xffffffffu);
+          if (lane == r) { sk = mu; si = wi; }
+          if (lane == (int)(wi & 31)) kr[wi] = 0;
+          __syncwarp();
+        }
+      } else {
+        lane_sort_desc<4>(key, id);
+        warp_select_lists<4>(key, id, k, lane, sk, si);
+      }
+      float sv = 0.0f;
+      if (lane < k) {
+        // select-only: the weight uses z, which this CTA stored (or the GEMM did)
+        const float zsel = select_bias ? z[(size_t)t * E + si] : f32_from_order_key(sk);
+        sv = 1.0f / (1.0f + expf(-zsel));
+      }
+      float ssum = 0.0f;
+      for (int r = 0; r < k; ++r) ssum += __shfl_sync(0xffffffffu, sv, r);
+      if (lane < k) {
+        idx_out[(size_t)t * k + lane] = (int)si;
+        w_out[(size_t)t * k + lane] = sv / ssum;
+      }
+    }
+    __syncthreads();
   }
-  __syncwarp();
 }
 
 // ---------------------------------------------------------------- combine

@@ -14,12 +14,10 @@
 // its fp32 partial to zpart[s].  Roles as in gemm.cuh: warp 0 loads (TMA), warp 1 issues
 // MMAs, warps 2..9 drain and store.
 //
-// Selection is fused: the CTA that completes the last split of a (token tile, expert tile)
-// adds the partials in split order plus the bias and writes z; the CTA that completes the
-// last expert tile of a token tile has every logit of those tokens and runs the sigmoid
-// top-k (topk_sigmoid_row_regs, or _smem for E > 1024) for them.  "Last" is decided by counters (atomicAdd after a
-// fence of the CTA's stores); nothing waits on another CTA, and the counters are zeroed
-// before the launch.
+// Selection runs in the next launch (route_select_kernel in kernels.cuh), which also sums
+// the split partials: a kernel boundary publishes the logits to it, where a selection fused
+// into this epilogue needs GPU-scope fences and counters between CTAs, which measured far
+// slower under this kernel's load.
 #pragma once
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -31,17 +29,10 @@ struct RouterArgs {
   int m_tiles;     // ceil(E / 128)
   int ksplit;      // K splits (1: no split)
   int chains_per;  // 64-column chains per split
-  const float* bias;        // logit bias added to z, or NULL
-  const float* sel_bias;    // select-only bias (selection key z + b), or NULL
-  float* z;        // [T][E] logits
+  const float* bias;        // logit bias added to z (ksplit == 1), or NULL
+  float* z;        // [T][E] logits (ksplit == 1)
   float* zpart;    // [ksplit][T][E] partials without bias (ksplit > 1)
   unsigned int* status;
-  int k;           // experts per token
-  int* idx;        // [T][k] selected experts, descending key
-  float* w;        // [T][k] renormalised sigmoid weights
-  int* cnt_split;  // [token tiles][m_tiles] splits done (zeroed before the launch)
-  int* cnt_tile;   // [token tiles] expert tiles done (zeroed before the launch)
-  int topk_warps;  // epilogue warps with an E-float selection row in shared memory
 };
 
 struct RouterTile {
@@ -66,7 +57,7 @@ struct RouterCfg {
   static constexpr int A_BYTES = 3 * A_PLANE;
   static constexpr int B_BYTES = RBN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;   // + topk rows (dynamic)
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
   static constexpr int TMEM_COLS = 2 * RBN <= 256 ? 256 : 512;
   static_assert(RBN % 64 == 0 && RBN <= 256, "RBN");
   static_assert(STAGE_BYTES % 1024 == 0, "alignment");
@@ -85,12 +76,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* pfull = empty_bar + STAGES;   // [2] partial buffer written
   uint64_t* pempty = pfull + 2;           // [2] partial buffer drained
   uint64_t* drain_bar = pempty + 2;
-  uint64_t* epi_bar = drain_bar + 1;      // the 8 epilogue warps meet here (fused selection)
-  uint32_t* tmem_holder = (uint32_t*)(epi_bar + 1);
+  uint32_t* tmem_holder = (uint32_t*)(drain_bar + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
   int* fills = (int*)(tmem_holder + 2);   // abort cleanup: [0] loads armed, [1] loads consumed
-  volatile int* last_flag = (volatile int*)(fills + 2);   // [2] fused-selection decisions
-  float* topk_rows = (float*)(smem + C::SMEM_BYTES - 1024);  // [topk_warps][E] after the control block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tok_tiles = (args.T + RBN - 1) / RBN;
@@ -106,7 +94,6 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(smem_u32(pempty + b), 8);
     }
     mbar_init(smem_u32(drain_bar), 1);
-    mbar_init(smem_u32(epi_bar), 8);
     *abort_flag = 0;
     fills[0] = fills[1] = 0;
     fence_mbar_init();
@@ -202,20 +189,6 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t g = 0;
     bool ok = true;
-    // Bounded meeting point of the 8 epilogue warps (an mbarrier phase per meeting), so that
-    // a warp that gives up cannot leave the others waiting; it also orders the shared-memory
-    // flags written before it.
-    uint32_t es_phase = 0;
-    auto epi_sync = [&]() -> bool {
-      bool r = true;
-      if (lane == 0) {
-        mbar_arrive(smem_u32(epi_bar));
-        r = mbar_wait(smem_u32(epi_bar), es_phase, args.status, abort_flag);
-      }
-      es_phase ^= 1u;
-      __syncwarp();
-      return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
-    };
     for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
       const RouterTile rt = router_tile(args, RBN, t);
       const int mt = rt.mt, row0 = rt.row0;
@@ -233,17 +206,18 @@ __global__ void __launch_bounds__(320, 1)
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
         tc_fence_after();
+        // all of this warp's chunks in flight, one wait: the drain keeps pace with the
+        // 12-MMA chain that refills the other buffer
+        uint32_t r[MYCH][16];
 #pragma unroll
-        for (int i = 0; i < MYCH; ++i) {
-          const int ch = cs * MYCH + i;
-          if (ch < nchunks) {
-            uint32_t r[16];
-            tmem_ld16(tmem_base + lane_off + b * RBN + ch * 16, r);
-            tmem_ld_wait();
+        for (int i = 0; i < MYCH; ++i)
+          if (cs * MYCH + i < nchunks) tmem_ld16(tmem_base + lane_off + b * RBN + (cs * MYCH + i) * 16, r[i]);
+        tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) accv[i][j] += __uint_as_float(r[j]);
-          }
-        }
+        for (int i = 0; i < MYCH; ++i)
+          if (cs * MYCH + i < nchunks)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) accv[i][j] += __uint_as_float(r[i][j]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(pempty + b));
@@ -261,80 +235,6 @@ __global__ void __launch_bounds__(320, 1)
             const int n = (cs * MYCH + i) * 16 + j;
             if (n < n_valid) out[(size_t)(row0 + n) * args.E + e] = split ? accv[i][j] : accv[i][j] + bias;
           }
-      }
-
-      // ---- fused selection (see the file comment)
-      const int tt = row0 / RBN;
-      __threadfence();                                 // this thread's stores, before the count
-      if (!(ok = epi_sync())) break;
-      if (warp == 2 && lane == 0) {
-        int last = 1;
-        if (split) {
-          int* c = args.cnt_split + (size_t)tt * args.m_tiles + mt;
-          last = atomicAdd(c, 1) == args.ksplit - 1;
-        }
-        last_flag[0] = last;
-      }
-      if (!(ok = epi_sync())) break;
-      if (!last_flag[0]) continue;
-      __threadfence();                                 // every split of this tile is visible
-      if (split) {
-        // z = the partials summed in split order, plus the logit bias.  The 256 epilogue
-        // threads walk the tile's (token, expert) elements flat (expert fastest, so a warp's
-        // loads are coalesced), four elements and eight partials at a time in flight.
-        const int et = (warp - 2) * 32 + lane;
-        const int nel = n_valid * 128;
-        const size_t plane = (size_t)args.T * args.E;
-        for (int i0 = et; i0 < nel; i0 += 4 * 256) {
-          size_t o[4];
-          bool in[4];
-          float v[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * 256;
-            const int ee = mt * 128 + (i & 127);
-            in[u] = i < nel && ee < args.E;
-            o[u] = in[u] ? (size_t)(row0 + (i >> 7)) * args.E + ee : 0;
-            v[u] = in[u] ? __ldcg(args.zpart + o[u]) : 0.0f;
-          }
-          for (int s0 = 1; s0 < args.ksplit; s0 += 8) {
-            float pp[4][8];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int q8 = 0; q8 < 8; ++q8)
-                pp[u][q8] = (in[u] && s0 + q8 < args.ksplit) ? __ldcg(args.zpart + (size_t)(s0 + q8) * plane + o[u]) : 0.0f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int q8 = 0; q8 < 8; ++q8)
-                if (s0 + q8 < args.ksplit) v[u] += pp[u][q8];
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (in[u]) args.z[o[u]] = args.bias ? v[u] + __ldg(args.bias + (int)(o[u] % args.E)) : v[u];
-        }
-      }
-      __threadfence();
-      if (!(ok = epi_sync())) break;
-      if (warp == 2 && lane == 0) last_flag[1] = atomicAdd(args.cnt_tile + tt, 1) == args.m_tiles - 1;
-      if (!(ok = epi_sync())) break;
-      if (!last_flag[1]) continue;
-      __threadfence();                                 // every logit of the token tile is visible
-      const int ew = warp - 2;
-      if (args.E <= 32 * kTopkKeysPerLane) {
-        for (int n = ew; n < n_valid; n += 8) {
-          const size_t t_ = (size_t)(row0 + n);
-          topk_sigmoid_row_regs(args.z + t_ * args.E, args.sel_bias, args.E, args.k, args.idx + t_ * args.k,
-                                args.w + t_ * args.k, lane);
-        }
-      } else if (ew < args.topk_warps) {
-        float* row = topk_rows + (size_t)ew * args.E;
-        for (int n = ew; n < n_valid; n += args.topk_warps) {
-          const size_t t_ = (size_t)(row0 + n);
-          topk_sigmoid_row_smem(args.z + t_ * args.E, args.sel_bias, args.E, args.k, row, args.idx + t_ * args.k,
-                                args.w + t_ * args.k, lane);
-        }
       }
     }
   }

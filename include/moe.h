@@ -136,10 +136,11 @@ moe_status_t moe_quant_mxfp8(const void* x_bf16, int rows, int cols, uint8_t* q_
  * z = x . W_r + bias (fp32-accurate: W_r is split into three bf16 terms on the tensor
  * cores), s = sigmoid(z); per token the k largest z in descending order (lower expert
  * index on ties) and w_j = s_j / sum of the selected s.  With MOE_BIAS_SELECT_ONLY the
- * bias enters only the selection key z + b (see moe_bias_mode_t).  One kernel (plus the
- * fp32 -> three-plane split of W_r, see MOE_FLAG_STATIC_ROUTER, and a memset of the
- * selection counters): the CTA that completes a token tile's last logit tile selects
- * its tokens' experts (a warp per token).
+ * bias enters only the selection key z + b (see moe_bias_mode_t).  Two kernels (plus the
+ * fp32 -> three-plane split of W_r, see MOE_FLAG_STATIC_ROUTER): the logit GEMM, then a
+ * selection kernel that sums the GEMM's K-split partials (when it split K) and selects
+ * in two stages inside each CTA: 8 warps each list a token's k best keys in one eighth
+ * of the experts, and one warp merges the 8 lists.
  * x_bf16: device [T][d]; W_r: device fp32 [d][E]; bias: device fp32 [E] or NULL;
  * idx: device int32 [T][k]; w: device fp32 [T][k]; logits_opt: device fp32 [T][E] or
  * NULL (receives z).  Uses the plan workspace. */

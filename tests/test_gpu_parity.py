@@ -439,14 +439,20 @@ def test_route_and_forward_replay_from_a_cuda_graph():
     assert case.plan.check()[0] == 0
 
 
-@pytest.mark.parametrize("E,k,select_only", [(96, 8, False), (1100, 16, False), (64, 4, True)])
-def test_route_exact_ties_lower_index_wins(E, k, select_only):
+@pytest.mark.parametrize("E,k,select_only,T", [(96, 8, False, 40), (600, 16, False, 40), (1100, 32, False, 40),
+                                                 (2100, 16, False, 40), (64, 4, True, 40), (300, 24, True, 40),
+                                                 (896, 16, False, 1301), (160, 32, True, 1301)])
+def test_route_exact_ties_lower_index_wins(E, k, select_only, T):
     """Exact ties in the selection key: duplicated router columns give equal logits, an
     all-zero token gives every expert the logit +0 (and -0 where the bias is -0), and in the
     select-only mode equal keys come from different (z, b) pairs.  The selection on the
-    GPU's own logits must equal the oracle's (descending key, lower index first), also with
-    more experts than the register form holds (E = 1100 takes the shared-memory form)."""
-    T, d = 40, 128
+    GPU's own logits must equal the oracle's (descending key, lower index first) for every
+    width of the selection kernel's first stage (1, 2, 4, 8 and 16 experts per lane: E up
+    to 256, 512, 1024, 2048, 4096), through both forms of its second stage (candidates
+    above the lane-maxima threshold; and, for the all-zero token, whose keys all tie, the
+    scan of every key), and with T = 1301 in 8-token groups, a ragged last group
+    included."""
+    d = 128
     g = torch.Generator().manual_seed(E + k)
     x = torch.randn((T, d), generator=g).to(torch.bfloat16)
     x[3] = 0.0
