@@ -24,15 +24,16 @@ namespace {
 //   an expert ~146 +- 12 rows, so 176 keeps all but a handful of experts in one tile (with
 //   160, one in eight was split in two half-full tiles, each costing as much tensor time as
 //   a full one);
-//   32 (default when T*k <= 8*E, decode): swap-AB with up to 32 token rows, 5 stages
-//   (38 KB): with a few tokens per expert the weight stream is the whole cost and the fifth
-//   stage keeps another 16 KB weight tile per SM in flight;
+//   32 (default when T*k <= 8*E, decode): swap-AB with up to 32 token rows, 6 stages
+//   (36 KB of tiles + 1.5 KB of scale atoms each, the whole 227 KB): with a few tokens per
+//   expert the weight stream is the whole cost, and each stage keeps another 16 KB weight
+//   tile per SM in flight (5 -> 4 stages measured 6% slower);
 //   128 (selectable): the WN orientation (gemm.cuh), token rows on M and 256 weight rows on
 //   N, 4 stages (50 KB).  Half the MMAs of swap-AB per weight byte, bit-identical results,
-//   but measured slower at every token count (see the design notes), so never the default.
+//   but measured slower at every token count, so never the default.
 constexpr int kBN = 176, kStages = 4;
 constexpr int kBNMid = 128, kStagesMid = 4;
-constexpr int kBNSmall = 32, kStagesSmall = 5;
+constexpr int kBNSmall = 32, kStagesSmall = 6;
 constexpr int kBNMin = kBNSmall;   // workspace sizing: the most tiles either configuration forms
 constexpr int kPermThreads = 256;
 constexpr int kRouterBN = 128;  // tokens per router tile
@@ -208,6 +209,25 @@ static void carve(moe_plan_s* p) {
   p->total = o;
 }
 
+// Launch with programmatic stream serialization: the kernel may start its prologue while
+// the previous kernel on the stream finishes; every kernel of the layer waits for that one
+// (griddep_wait) before its first global memory access.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // cudaFuncSetAttribute acts on the current device: remember, per kernel and per device
 // (bit d of `done`), which ones already had their dynamic shared-memory limit raised.
 template <class K>
@@ -230,8 +250,7 @@ static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, con
   const cudaError_t e = ensure_smem_attr(kern, Cfg::SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s>>>(a, tA, tB);
-  return cudaGetLastError();
+  return launch_k(kern, grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s, a, tA, tB);
 }
 
 // Routed (block-scaled) GEMMs: the three configurations above.  Dense (bf16) GEMMs:
@@ -281,11 +300,11 @@ static cudaError_t run_permute(moe_plan_s* p, const int32_t* idx, int T, int bn,
   if (set_smem_attrs() != cudaSuccess) return cudaErrorInvalidValue;
   const int nch = p->nchunks(T);
   int* chunk = p->at<int>(p->o_chunk);
-  perm_histogram_kernel<<<nch, 256, p->E * 4, s>>>(idx, T, p->k, p->E, p->tokens_per_chunk(), chunk,
+  launch_k(perm_histogram_kernel, nch, 256, p->E * 4, s, idx, T, p->k, p->E, p->tokens_per_chunk(), chunk,
                                                    p->at<unsigned int>(p->o_status));
-  perm_scan_kernel<<<1, 1024, (2 * p->E + 32) * 4, s>>>(chunk, nch, p->E, bn, p->at<int>(p->o_counts),
+  launch_k(perm_scan_kernel, 1, 1024, (2 * p->E + 32) * 4, s, chunk, nch, p->E, bn, p->at<int>(p->o_counts),
                                                          p->at<int>(p->o_offsets), p->at<int>(p->o_tiles));
-  perm_place_kernel<<<nch, kPermThreads, (kPermThreads / 32) * p->E * 4, s>>>(
+  launch_k(perm_place_kernel, nch, kPermThreads, (kPermThreads / 32) * p->E * 4, s,
       idx, T, p->k, p->E, p->tokens_per_chunk(), chunk, p->at<int>(p->o_perm), p->at<int>(p->o_inv));
   return cudaGetLastError();
 }
@@ -421,7 +440,7 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   if (!aligned(z, 16)) return MOE_ERR_ALIGNMENT;
   if (!(p->flags & MOE_FLAG_STATIC_ROUTER) || p->planes_of != (const void*)W_r) {
     p->prof.begin(MOE_STAGE_ROUTER_SPLIT, s);
-    router_split_kernel<<<dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s>>>(W_r, d, E, planes);
+    launch_k(router_split_kernel, dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s, W_r, d, E, planes);
     p->prof.end(s);
     p->planes_of = W_r;
   }
@@ -472,7 +491,7 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     if (ensure_smem_attr(kern, RC::SMEM_BYTES, router_done) != cudaSuccess) return MOE_ERR_CUDA;
     const int tiles = base_tiles * ra.ksplit;
     p->prof.begin(MOE_STAGE_ROUTER_GEMM, s);
-    kern<<<std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s>>>(ra, tA, tB);
+    launch_k(kern, std::min(tiles, p->num_sms), 320, RC::SMEM_BYTES, s, ra, tA, tB);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     p->prof.end(s);
   }
@@ -489,7 +508,7 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
     cudaError_t err = cudaSuccess;
     auto launch = [&](auto kern, std::atomic<uint64_t>& done) {
       err = ensure_smem_attr(kern, 8 * kMaxExperts * 4, done);
-      if (err == cudaSuccess) kern<<<grid, 256, smem, s>>>(ra.zpart, ra.ksplit, plane, lbias, sel, z, T, E, k, tpc, idx, w);
+      if (err == cudaSuccess) launch_k(kern, grid, 256, smem, s, ra.zpart, ra.ksplit, plane, lbias, sel, z, T, E, k, tpc, idx, w);
     };
     static std::atomic<uint64_t> sel_done[5];
     p->prof.begin(MOE_STAGE_TOPK, s);
@@ -561,7 +580,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     __nv_bfloat16* xn = p->at<__nv_bfloat16>(p->o_xn);
     p->prof.begin(MOE_STAGE_LATENT_IN, s);
     if (dense_bf16_f32(p, lat->w_down, de, x, d, T, xl, dbn, s) != cudaSuccess) return MOE_ERR_CUDA;
-    rmsnorm_bf16_kernel<<<T, 256, 0, s>>>(xl, lat->gamma, de, p->eps_lat, xn);
+    launch_k(rmsnorm_bf16_kernel, T, 256, 0, s, xl, lat->gamma, de, p->eps_lat, xn);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     xin = xn;
@@ -578,10 +597,10 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     const long long n = (long long)T * (de / 32);
     p->prof.begin(MOE_STAGE_QUANT, s);
     uint8_t* xs_tok = p->at<uint8_t>(p->o_xs_tok);
-    quant_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+    launch_k(quant_scatter_kernel, (unsigned)((n + 255) / 256), 256, 0, s,
         (const uint16_t*)xin, T, de, k, p->at<int>(p->o_inv), A, xq, xs_tok);
     const int max_gt = A / bn + E + 1;   // bound on the group-tiles of this call
-    scale_tiles_kernel<<<max_gt, 256, 0, s>>>(xs_tok, de / 32, p->at<int>(p->o_perm), p->at<int>(p->o_counts),
+    launch_k(scale_tiles_kernel, max_gt, 256, 0, s, xs_tok, de / 32, p->at<int>(p->o_perm), p->at<int>(p->o_counts),
                                               p->at<int>(p->o_offsets), p->at<int>(p->o_tiles), E, de / 128, xs);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -682,9 +701,9 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
         return MOE_ERR_CUDA;
       const long long n = (long long)T * Is;
       if (p->act == MOE_ACT_CLAMPED_SWIGLU)
-        split_glu_reduce_kernel<1><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_gu, T, Is, a.split_stride, hsh);
+        launch_k(split_glu_reduce_kernel<1>, (unsigned)((n + 255) / 256), 256, 0, s, spart, ks_gu, T, Is, a.split_stride, hsh);
       else
-        split_glu_reduce_kernel<0><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_gu, T, Is, a.split_stride, hsh);
+        launch_k(split_glu_reduce_kernel<0>, (unsigned)((n + 255) / 256), 256, 0, s, spart, ks_gu, T, Is, a.split_stride, hsh);
       if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       const cudaError_t e = p->act == MOE_ACT_CLAMPED_SWIGLU
@@ -721,7 +740,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
       if (launch_gemm<KIND_BF16, EPI_F32>(dbn, b, tA2, tB2, std::min(tiles * ks_dn, p->num_sms), s) != cudaSuccess)
         return MOE_ERR_CUDA;
       const long long n = (long long)T * d;
-      split_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(spart, ks_dn, n, b.split_stride, ys);
+      launch_k(split_sum_kernel, (unsigned)((n + 255) / 256), 256, 0, s, spart, ks_dn, n, b.split_stride, ys);
       if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       if (launch_gemm<KIND_BF16, EPI_F32>(dbn, b, tA2, tB2, std::min(tiles, p->num_sms), s) != cudaSuccess)
@@ -735,7 +754,7 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
   if (!lat) {
     // a9: weighted combine with the shared output
     p->prof.begin(MOE_STAGE_COMBINE, s);
-    combine_kernel<<<dim3(T, (d + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
+    launch_k(combine_kernel, dim3(T, (d + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s,
         O, ys, w, p->at<int>(p->o_inv), T, d, k, (__nv_bfloat16*)y);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -744,13 +763,13 @@ static moe_status_t forward_impl(moe_plan_t p, const void* x, int T, const int32
     __nv_bfloat16* yl = p->at<__nv_bfloat16>(p->o_yl);
     float* yr = p->at<float>(p->o_yr);
     p->prof.begin(MOE_STAGE_COMBINE, s);
-    combine_kernel<<<dim3(T, (de + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s>>>(
+    launch_k(combine_kernel, dim3(T, (de + kCombineCols - 1) / kCombineCols), kCombineThreads, k * 8, s,
         O, nullptr, w, p->at<int>(p->o_inv), T, de, k, yl);
     p->prof.end(s);
     p->prof.begin(MOE_STAGE_LATENT_OUT, s);
     if (dense_bf16_f32(p, lat->w_up, d, yl, de, T, yr, dbn, s) != cudaSuccess) return MOE_ERR_CUDA;
     const long long n = (long long)T * d;
-    add_bf16_kernel<<<(unsigned)((n / 4 + 255) / 256), 256, 0, s>>>(yr, ys, n, (__nv_bfloat16*)y);
+    launch_k(add_bf16_kernel, (unsigned)((n / 4 + 255) / 256), 256, 0, s, yr, ys, n, (__nv_bfloat16*)y);
     p->prof.end(s);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }

@@ -94,12 +94,18 @@ struct GemmCfg {
   static constexpr int BK = KIND == KIND_MX ? 128 : 64;        // elements per K tile (128 B rows)
   static constexpr int A_BYTES = BM * 128;                     // smem (FP4 padded to 1 B/elem)
   static constexpr int B_BYTES = BN_MAX * 128;
-  static constexpr int SFA_BYTES = KIND == KIND_MX ? 1024 : 0;
+  static constexpr int SFA_BYTES = KIND == KIND_MX ? 1024 : 0;   // two 512 B atoms
   static constexpr int SFB_ATOMS = (BN_MAX + 127) / 128;
-  static constexpr int SFB_BYTES = KIND == KIND_MX ? 1024 : 0;   // room for two 512 B atoms
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int SFB_BYTES = KIND == KIND_MX ? SFB_ATOMS * 512 : 0;
+  // Shared memory: the stages' A and B tiles (1024-byte aligned for the swizzled layouts),
+  // then every stage's scale atoms, then the control block.  Keeping the small scale atoms
+  // out of the tile stride lets the 32-row configuration hold six stages.
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int CTRL_OFFSET = SF_OFFSET + STAGES * SF_STAGE_BYTES;
   static constexpr int A_TX = KIND == KIND_MX ? BM * BK / 2 : BM * BK * 2;  // global bytes
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+  static constexpr int SMEM_BYTES = CTRL_OFFSET + 1024 /*barriers*/ + 1024 /*align*/;
   // scale factors in TMEM, one 16-column buffer per pipeline stage:
   //   weights: 4 columns per 128-row half (+0, +4), tokens: 4 columns per 128 rows (+8, +12)
   // after the accumulator (two halves of BN_MAX columns, or WN: 256 columns)
@@ -110,6 +116,7 @@ struct GemmCfg {
   static_assert(SFB_ATOMS <= 2, "scale buffer holds two B atoms");
   static_assert(TMEM_SF + 16 * STAGES <= TMEM_COLS, "TMEM budget");
   static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(SF_STAGE_BYTES % 128 == 0, "scale atom alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // WN: the M=128 MMA reads 128 token rows (16 KB) from the token region whatever the
   // tile's row count, so the region must hold 128 rows (rows past the tile's are stale and
@@ -179,6 +186,8 @@ __device__ __forceinline__ float glu_f(float g, float u);
 template <int ACT>
 __global__ void split_glu_reduce_kernel(const float* __restrict__ part, int nsplit, int T, int I,
                                         long long split_stride, __nv_bfloat16* __restrict__ h) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)T * I) return;
   const int t = (int)(i / I), c = (int)(i - (long long)t * I);
@@ -195,6 +204,8 @@ __global__ void split_glu_reduce_kernel(const float* __restrict__ part, int nspl
 // out[i] = sum over s, in order, of part[s * split_stride + i].
 __global__ void split_sum_kernel(const float* __restrict__ part, int nsplit, long long n, long long split_stride,
                                  float* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float v = 0.0f;
@@ -239,7 +250,7 @@ __global__ void __launch_bounds__(384, 1)
   using C = GemmCfg<KIND, BN_MAX, STAGES, WN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* ctrl = smem + STAGES * C::STAGE_BYTES;
+  uint8_t* ctrl = smem + C::CTRL_OFFSET;
   uint64_t* full_bar = (uint64_t*)ctrl;
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* sf_full = empty_bar + STAGES;        // scale blocks of the stage are in smem
@@ -285,6 +296,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the prologue above touches no global memory; the previous kernel's results are read
+  // (and buffers it may still read are written) only after this
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int num_tiles = gemm_num_tiles(args, BN_MAX);
 
@@ -339,7 +354,7 @@ __global__ void __launch_bounds__(384, 1)
                   args.sfa + (((size_t)ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * 1024;
               asm volatile(
                   "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], 1024, [%2];" ::
-                      "r"(smem_u32(sA + C::A_BYTES + C::B_BYTES)),
+                      "r"(smem_u32(smem + C::SF_OFFSET + stage * C::SF_STAGE_BYTES)),
                   "l"(sfa_src), "r"(sb)
                   : "memory");
             }
@@ -383,7 +398,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint8_t* src = args.sfb + ((size_t)ti.gt * args.k_tiles + kt) * SF_TILE_BYTES;
             asm volatile(
                 "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-                    "r"(smem_u32(sB + C::B_BYTES + C::SFA_BYTES)),
+                    "r"(smem_u32(smem + C::SF_OFFSET + stage * C::SF_STAGE_BYTES + C::SFA_BYTES)),
                 "l"(src), "r"(sfb_bytes), "r"(sb)
                 : "memory");
           }
@@ -403,7 +418,7 @@ __global__ void __launch_bounds__(384, 1)
     // refilling, i.e. after the MMAs that read it committed.
     if (KIND == KIND_MX && lane == 0) {
       // no-swizzle descriptor of stage 0's A scale atoms (32 rows x 16 B, 128 B per 8 rows)
-      const uint64_t sf_desc0 = smem_desc(smem_u32(smem) + C::A_BYTES + C::B_BYTES, 16, 128, 0);
+      const uint64_t sf_desc0 = smem_desc(smem_u32(smem) + C::SF_OFFSET, 16, 128, 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -418,7 +433,7 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           ++nfill;
           tc_fence_after();
-          const uint64_t sfa_desc = sf_desc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t sfa_desc = sf_desc0 + (uint64_t)((stage * C::SF_STAGE_BYTES) >> 4);
           const uint64_t sfb_desc = sfa_desc + (uint64_t)(C::SFA_BYTES >> 4);
           const uint32_t tsf = tmem_base + C::TMEM_SF + 16 * stage;
           tc_cp_32x128b_warpx4(tsf, sfa_desc);

@@ -84,6 +84,8 @@ __global__ void quant_mxfp8_kernel(const uint16_t* __restrict__ x, int rows, int
 __global__ void quant_scatter_kernel(const uint16_t* __restrict__ x, int T, int cols, int k,
                                      const int* __restrict__ inv, int A_rows,
                                      uint8_t* __restrict__ xq, uint8_t* __restrict__ xs_tok) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int nb = cols >> 5;
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= (long long)T * nb) return;
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(256)
     scale_tiles_kernel(const uint8_t* __restrict__ xs_tok, int nb, const int* __restrict__ perm_tok,
                        const int* __restrict__ counts, const int* __restrict__ offsets,
                        const int* __restrict__ tile_prefix, int E, int k_tiles, uint8_t* __restrict__ xs) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int gt = blockIdx.x;
   if (gt >= __ldg(tile_prefix + E)) return;
   int lo = 0, hi = E - 1;   // last group whose first tile is <= gt
@@ -177,6 +181,8 @@ __global__ void __launch_bounds__(256)
 __global__ void perm_histogram_kernel(const int* __restrict__ idx, int T, int k, int E,
                                       int tokens_per_chunk, int* __restrict__ chunk_counts,
                                       unsigned int* status) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -236,6 +242,8 @@ __device__ void block_exclusive_scan(int* vals, int n, int* warp_tot) {
 __global__ void perm_scan_kernel(int* __restrict__ chunk_counts, int nchunks, int E, int bn_max,
                                  int* __restrict__ counts, int* __restrict__ offsets,
                                  int* __restrict__ tile_prefix) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ int sh[];
   int* s_off = sh;            // E
   int* s_tiles = sh + E;      // E
@@ -275,6 +283,8 @@ __global__ void perm_scan_kernel(int* __restrict__ chunk_counts, int nchunks, in
 __global__ void perm_place_kernel(const int* __restrict__ idx, int T, int k, int E,
                                   int tokens_per_chunk, const int* __restrict__ chunk_base,
                                   int* __restrict__ perm_tok, int* __restrict__ inv) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ uint32_t masks[];  // [warps][E]
   const int warps = blockDim.x >> 5;
   for (int i = threadIdx.x; i < warps * E; i += blockDim.x) masks[i] = 0;
@@ -377,6 +387,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
                                                            const float* __restrict__ select_bias, float* z, int T,
                                                            int E, int k, int tpc, int* __restrict__ idx_out,
                                                            float* __restrict__ w_out) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ uint32_t sel_keys[];   // [tpc][E] order keys
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int t0 = blockIdx.x * tpc; t0 < T; t0 += gridDim.x * tpc) {
@@ -497,6 +509,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const __nv_bfloat16* __restrict__ O, const float* __restrict__ ys,
                    const float* __restrict__ w, const int* __restrict__ inv, int T, int d, int k,
                    __nv_bfloat16* __restrict__ y) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int t = blockIdx.x;
   extern __shared__ int s_inv[];
   float* s_w = (float*)(s_inv + k);
@@ -551,6 +565,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 __global__ void __launch_bounds__(256)
     rmsnorm_bf16_kernel(const float* __restrict__ xl, const float* __restrict__ gamma, int cols, float eps,
                         __nv_bfloat16* __restrict__ xn) {
+  griddep_wait();
+  griddep_launch_dependents();
   const float* row = xl + (size_t)blockIdx.x * cols;
   float ss = 0.0f;
   for (int c = threadIdx.x; c < cols; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
@@ -570,6 +586,8 @@ __global__ void __launch_bounds__(256)
 // y = bf16(a + b) (b may be NULL), fp32 inputs, 4 elements per thread (n % 4 == 0).
 __global__ void add_bf16_kernel(const float* __restrict__ a, const float* __restrict__ b, long long n,
                                 __nv_bfloat16* __restrict__ y) {
+  griddep_wait();
+  griddep_launch_dependents();
   const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i >= n) return;
   float4 v = __ldg((const float4*)(a + i));
@@ -654,6 +672,8 @@ __global__ void pack_mxfp4_kernel(const float* __restrict__ src0, const float* _
 // W = hi + mid + lo exactly (hi = bf16(W), mid = bf16(W - hi), lo = bf16(W - hi - mid)).
 __global__ void router_split_kernel(const float* __restrict__ W, int d, int E,
                                     __nv_bfloat16* __restrict__ planes) {
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float tile[32][33];
   const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {

@@ -118,6 +118,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(map), "r"(bar), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the previous
+// kernel on the stream has finished.  griddep_wait() blocks until that kernel has completed
+// and its memory operations are visible; every kernel of the layer calls it before its first
+// global memory access (read or write), so only prologue work (barrier setup, TMEM
+// allocation, tensor-map prefetch) overlaps the previous kernel's tail.  Without a
+// programmatic dependency both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream begin launching (its CTAs still wait in griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Bring a tensor tile into L2 without touching shared memory (no completion tracking).
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)

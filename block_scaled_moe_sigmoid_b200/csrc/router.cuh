@@ -108,6 +108,10 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the prologue above touches no global memory; the previous kernel's results are read
+  // (and buffers it may still read are written) only after this
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------- loads

@@ -277,7 +277,7 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  *   this many K tiles ahead of the shared-memory loads (0..64, 0 = off).
  * MOE_OPT_PREFETCH_B: accepted and ignored (reserved).
  * MOE_OPT_TILE_N: token rows per routed grouped-GEMM tile.  0 (default) picks per call:
- *   32 rows (5-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure
+ *   32 rows (6-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure
  *   weight stream, else 176 rows (4 stages); both put 256 weight rows on the MMA's M side
  *   and the token rows on its N side.  128 selects the other orientation: token rows on M
  *   (up to 128 per tile) and 256 weight rows on N.  32, 128 or 176 forces one
