@@ -440,7 +440,7 @@ moe_status_t moe_route(moe_plan_t p, const void* x, int T, const float* W_r, con
   if (!aligned(z, 16)) return MOE_ERR_ALIGNMENT;
   if (!(p->flags & MOE_FLAG_STATIC_ROUTER) || p->planes_of != (const void*)W_r) {
     p->prof.begin(MOE_STAGE_ROUTER_SPLIT, s);
-    launch_k(router_split_kernel, dim3((E + 31) / 32, (d + 31) / 32), dim3(32, 8), 0, s, W_r, d, E, planes);
+    launch_k(router_split_kernel, dim3((E + 31) / 32, (d + 63) / 64), dim3(256), 0, s, W_r, d, E, planes);
     p->prof.end(s);
     p->planes_of = W_r;
   }

@@ -670,31 +670,38 @@ __global__ void pack_mxfp4_kernel(const float* __restrict__ src0, const float* _
 
 // Router weights W_r fp32 [d][E] -> three bf16 planes W^T [E][3d] with
 // W = hi + mid + lo exactly (hi = bf16(W), mid = bf16(W - hi), lo = bf16(W - hi - mid)).
-__global__ void router_split_kernel(const float* __restrict__ W, int d, int E,
-                                    __nv_bfloat16* __restrict__ planes) {
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ W, int d, int E,
+                                                           __nv_bfloat16* __restrict__ planes) {
   griddep_wait();
   griddep_launch_dependents();
-  __shared__ float tile[32][33];
-  const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int i = i0 + r, e = e0 + threadIdx.x;
-    tile[r][threadIdx.x] = (i < d && e < E) ? W[(size_t)i * E + e] : 0.0f;
+  // block: 32 experts x 64 rows of W; coalesced 128-byte row reads, then per expert 64
+  // consecutive K elements of each plane as bf16 pairs (128-byte warp stores)
+  __shared__ float tile[64][33];
+  const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 64;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 8 warps
+  for (int r = ty; r < 64; r += 8) {
+    const int i = i0 + r, e = e0 + tx;
+    tile[r][tx] = (i < d && e < E) ? W[(size_t)i * E + e] : 0.0f;
   }
   __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int e = e0 + r, i = i0 + threadIdx.x;
-    if (e < E && i < d) {
-      const float w = tile[threadIdx.x][r];
+  for (int c = ty; c < 32; c += 8) {
+    const int e = e0 + c, i = i0 + 2 * tx;
+    if (e >= E || i >= d) continue;   // d is even (a multiple of 128)
+    __nv_bfloat162 p[3];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float w = tile[2 * tx + u][c];
       const __nv_bfloat16 hi = __float2bfloat16_rn(w);
       const float r1 = w - __bfloat162float(hi);
       const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
       const float r2 = r1 - __bfloat162float(mid);
       const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-      __nv_bfloat16* row = planes + (size_t)e * 3 * d;
-      row[i] = hi;
-      row[d + i] = mid;
-      row[2 * d + i] = lo;
+      if (u == 0) { p[0].x = hi; p[1].x = mid; p[2].x = lo; }
+      else        { p[0].y = hi; p[1].y = mid; p[2].y = lo; }
     }
+    __nv_bfloat16* row = planes + (size_t)e * 3 * d;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) *(__nv_bfloat162*)(row + (size_t)q * d + i) = p[q];
   }
 }
 
