@@ -342,12 +342,9 @@ __global__ void __launch_bounds__(384, 1)
           if (ok) {
             uint8_t* sA = smem + stage * C::STAGE_BYTES;
             const uint32_t fb = smem_u32(full_bar + stage);
-            mbar_arrive_expect_tx(fb, C::A_TX);
-            if constexpr (KIND == KIND_MX)   // tile-major weights: one contiguous 16 KB block
-              tma_load_2d(smem_u32(sA), &tmA, fb, 0, ((ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * C::BM, pol_a);
-            else
-              tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
             if constexpr (KIND == KIND_MX) {
+              // the scale atoms first: the scale warp's copies into TMEM then run while the
+              // large tile is still landing
               const uint32_t sb = smem_u32(sf_full + stage);
               mbar_arrive_expect_tx(sb, C::SFA_BYTES);
               const uint8_t* sfa_src =
@@ -358,6 +355,11 @@ __global__ void __launch_bounds__(384, 1)
                   "l"(sfa_src), "r"(sb)
                   : "memory");
             }
+            mbar_arrive_expect_tx(fb, C::A_TX);
+            if constexpr (KIND == KIND_MX)   // tile-major weights: one contiguous 16 KB block
+              tma_load_2d(smem_u32(sA), &tmA, fb, 0, ((ti.grp * args.m_tiles + ti.mt) * args.k_tiles + kt) * C::BM, pol_a);
+            else
+              tma_load_2d(smem_u32(sA), &tmA, fb, kt * C::BK, a_row, pol_a);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -389,8 +391,6 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t fb = smem_u32(full_bar + stage);
         if (lane == 0) {
           stage_n[stage] = ti.n_mma;
-          mbar_arrive_expect_tx(fb, nB * BOX_ROWS * 128);
-          tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
           if constexpr (KIND == KIND_MX) {
             const int sfb_bytes = ((ti.n_mma + 127) >> 7) * 512;
             const uint32_t sb = smem_u32(sf_full + stage);
@@ -402,6 +402,8 @@ __global__ void __launch_bounds__(384, 1)
                 "l"(src), "r"(sfb_bytes), "r"(sb)
                 : "memory");
           }
+          mbar_arrive_expect_tx(fb, nB * BOX_ROWS * 128);
+          tma_load_2d(smem_u32(sB), &tmB.box[nB - 1], fb, (kt % args.kb_wrap) * C::BK, ti.row0, pol_b);
         }
         __syncwarp();
         ++nfill;

@@ -23,7 +23,10 @@
  *   - Matrices are row-major.  Weights are stored out x in (row = output channel).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL = legacy
  *     default stream); none synchronises the host except moe_plan_check and
- *     moe_plan_stage_ms.
+ *     moe_plan_stage_ms.  The layer's kernels are launched with programmatic stream
+ *     serialization: each may start its prologue while the previous kernel on the stream
+ *     finishes, but touches no global memory before that kernel has completed, so stream
+ *     order holds for the caller's work before and after as usual.
  *   - Errors are returned as moe_status_t; nothing is thrown.  Argument checks happen
  *     before any launch, so an error return leaves outputs untouched.
  *   - Device-side faults (an out-of-range expert id, a pipeline wait that timed out) are
