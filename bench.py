@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode (T=64) measurement that the default workload adds")
-    ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 128, 176],
+    ap.add_argument("--tile-n", type=int, default=0, choices=[0, 32, 128, 160, 176],
                     help="grouped-GEMM token rows per tile (0 = the library's per-call choice)")
     return ap.parse_args()
 

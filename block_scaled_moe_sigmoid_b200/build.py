@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_sm100.so")
 SOURCES = ["api.cu"]
-DEPS = ["api.cu", "gemm.cuh", "kernels.cuh", "ptx.cuh", "router.cuh", "tiling.cuh"]
+DEPS = ["api.cu", "gemm.cuh", "gemm_pair.cuh", "kernels.cuh", "ptx.cuh", "router.cuh", "tiling.cuh"]
 HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
 
 NVCC_FLAGS = [

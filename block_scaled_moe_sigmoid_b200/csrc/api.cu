@@ -11,6 +11,7 @@
 
 #include "../../include/moe.h"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "kernels.cuh"
 #include "router.cuh"
 
@@ -33,6 +34,7 @@ namespace {
 //   but measured slower at every token count, so never the default.
 constexpr int kBN = 176, kStages = 4;
 constexpr int kBNMid = 128, kStagesMid = 4;
+constexpr int kBNPair = 160, kStagesPair = 5;   // CTA-pair configuration (gemm_pair.cuh)
 constexpr int kBNSmall = 32, kStagesSmall = 6;
 constexpr int kBNMin = kBNSmall;   // workspace sizing: the most tiles either configuration forms
 constexpr int kPermThreads = 256;
@@ -137,7 +139,7 @@ struct moe_plan_s {
   int bias_mode = MOE_BIAS_LOGIT;
   int flags = 0;
   const void* planes_of = nullptr;   // W_r the router planes were last split from
-  int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32, 128 or 176
+  int tile_n_opt = 0;         // MOE_OPT_TILE_N: 0 = automatic, else 32, 128, 160 or 176
   int last_bn = 0;            // token rows per tile in the last moe_forward
   int last_ksplit = 0;        // router K splits in the last moe_route
   int last_shared_split = 0;     // shared-expert gate/up K splits in the last moe_forward
@@ -253,13 +255,60 @@ static cudaError_t launch_gemm_cfg(const GemmArgs& a, const CUtensorMap& tA, con
   return launch_k(kern, grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, s, a, tA, tB);
 }
 
-// Routed (block-scaled) GEMMs: the three configurations above.  Dense (bf16) GEMMs:
+// The CTA-pair routed GEMM: clusters of two CTAs (grid rounded down to an even number of
+// SMs), programmatic stream serialization as for the other launches.
+template <int EPI>
+static cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
+                                   cudaStream_t s) {
+  using Cfg = PairCfg<kBNPair, kStagesPair>;
+  auto kern = gemm_pair_kernel<EPI, kBNPair, kStagesPair>;
+  static std::atomic<uint64_t> attr_done{0};
+  const cudaError_t e = ensure_smem_attr(kern, Cfg::SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(Cfg::NUM_THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // The kernel is persistent: every pair must be resident at once, and pairs of SMs that
+  // each hold a 222 KB CTA must share a GPC, so fewer pairs than SMs / 2 may fit.
+  static std::atomic<int> max_pairs_cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  int max_pairs = dev < 64 ? max_pairs_cache[dev].load(std::memory_order_acquire) : 0;
+  if (max_pairs <= 0) {
+    cfg.gridDim = dim3(grid & ~1);
+    if (cudaOccupancyMaxActiveClusters(&max_pairs, kern, &cfg) != cudaSuccess || max_pairs <= 0) return cudaErrorInvalidConfiguration;
+    if (dev < 64) max_pairs_cache[dev].store(max_pairs, std::memory_order_release);
+  }
+  grid = std::min(grid & ~1, 2 * max_pairs);
+  if (grid <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(grid);
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, a, tA, tB);
+}
+
+// Routed (block-scaled) GEMMs: the configurations above.  Dense (bf16) GEMMs:
 // swap-AB with 32 or 176 token rows (128 is only ever asked for the routed ones).
 template <int KIND, int EPI>
 static cudaError_t launch_gemm(int bn, const GemmArgs& a, const CUtensorMap& tA, const BMaps& tB, int grid,
                                cudaStream_t s) {
   if constexpr (KIND == KIND_MX) {
     if (bn == kBNMid) return launch_gemm_cfg<KIND, EPI, kBNMid, kStagesMid, true>(a, tA, tB, grid, s);
+    if (bn == kBNPair) {
+      // pairs of 256-row m-tiles; an odd m-tile count runs the same tiles on single CTAs
+      if (a.dense_rows < 0 && a.m_tiles % 2 == 0 && a.M_total % 256 == 0)
+        return launch_gemm_pair<EPI>(a, tA, tB, grid, s);
+      return launch_gemm_cfg<KIND, EPI, kBNPair, 4>(a, tA, tB, grid, s);
+    }
   }
   if (bn == kBNSmall) return launch_gemm_cfg<KIND, EPI, kBNSmall, kStagesSmall>(a, tA, tB, grid, s);
   return launch_gemm_cfg<KIND, EPI, kBN, kStages>(a, tA, tB, grid, s);
@@ -908,7 +957,8 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int option, int value) {
       p->pf_b = value != 0;
       return MOE_OK;
     case MOE_OPT_TILE_N:
-      if (value != 0 && value != kBNSmall && value != kBNMid && value != kBN) return MOE_ERR_INVALID_ARG;
+      if (value != 0 && value != kBNSmall && value != kBNMid && value != kBNPair && value != kBN)
+        return MOE_ERR_INVALID_ARG;
       p->tile_n_opt = value;
       return MOE_OK;
   }

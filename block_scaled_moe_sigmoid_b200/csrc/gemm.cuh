@@ -243,6 +243,116 @@ struct BMaps {
   CUtensorMap box[MAX_BOX];
 };
 
+// Swap-AB epilogue of one tile (accumulator lanes = output channels, columns = tokens):
+// warps 2..9, lane quarter q, column half `sub`.  release_tmem() hands the accumulator back
+// to the MMA issuer as soon as this warp has read what it needs.
+template <int KIND, int EPI, int BN_MAX, class Release>
+__device__ __forceinline__ void epilogue_swapab(const GemmArgs& args, const TileInfo& ti, uint32_t lane_base, int q,
+                                                int sub, int lane, Release&& release_tmem) {
+  const int nchunks = ti.n_mma >> 4;
+  constexpr int CH = BN_MAX / 16;
+  if constexpr (EpiTraits<EPI>::glu) {
+    // a = glu(g, u) for this warp's chunks (c = sub + 2 i) straight out of TMEM;
+    // TMEM goes back to the MMA warp before the quantisation and stores.
+    constexpr int CH2 = (CH + 1) / 2;   // this warp's chunks: c = sub + 2 i
+    float a[CH2][16];
+#pragma unroll
+    for (int i = 0; i < CH2; ++i) {
+      const int c = sub + 2 * i;
+      if (c < nchunks) {
+        uint32_t g[16], u[16];
+        tmem_ld16(lane_base + c * 16, g);
+        tmem_ld16(lane_base + BN_MAX + c * 16, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) a[i][j] = glu_f<EpiTraits<EPI>::act>(__uint_as_float(g[j]), __uint_as_float(u[j]));
+      }
+    }
+    release_tmem();
+    const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
+#pragma unroll
+    for (int i = 0; i < CH2; ++i) {
+      const int c = sub + 2 * i;
+      if (c >= nchunks) break;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int n = c * 16 + j;
+        if (n >= ti.n_valid) break;
+        const size_t row = (size_t)(ti.row0 + n);
+        if constexpr (EpiTraits<EPI>::mx8_out) {
+          const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a[i][j]) & 0x7FFFFFFFu);
+          const int e = mx_exp_e4m3(amax);
+          const float qv = a[i][j] * __uint_as_float((uint32_t)(127 - e) << 23);
+          const uint32_t code = f32x2_to_e4m3x2(qv, 0.0f) & 0xFFu;
+          ((uint8_t*)args.out0)[row * args.ld_out + ch] = (uint8_t)code;
+          if (lane == 0)   // scale byte for the down GEMM: K tile mt, block q, tile-major
+            ((uint8_t*)args.out1)[((size_t)ti.gt * args.m_tiles + ti.mt) * SF_TILE_BYTES +
+                                  sf_atom_offset(n) + q] = (uint8_t)(e + 127);
+        } else {
+          ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a[i][j]);
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_BF16) {
+    // round to bf16 pairs while draining TMEM, release it, then store
+    const int h = sub;
+    const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
+    uint32_t v[CH][8];
+    if (half_ok) {
+#pragma unroll
+      for (int c = 0; c < CH; ++c)
+        if (c < nchunks) {
+          uint32_t r[16];
+          tmem_ld16(lane_base + h * BN_MAX + c * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat162 p2 =
+                __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            v[c][j] = *(const uint32_t*)&p2;
+          }
+        }
+    }
+    release_tmem();
+    const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
+    if (half_ok && ch < args.M_total) {
+      uint16_t* out = (uint16_t*)args.out0;
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        if (c >= nchunks) break;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c * 16 + j;
+          if (n >= ti.n_valid) break;
+          out[(size_t)(ti.row0 + n) * args.ld_out + ch] = (uint16_t)(v[c][j >> 1] >> ((j & 1) * 16));
+        }
+      }
+    }
+  } else {
+    // fp32 results: store straight from TMEM chunk by chunk, release at the end
+    const int h = sub;
+    const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
+    const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
+    if (half_ok) {
+      const bool ch_ok = ch < args.M_total;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + h * BN_MAX + c * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c * 16 + j;
+          if (n >= ti.n_valid) break;
+          if (!ch_ok) continue;
+          ((float*)args.out0)[(size_t)ti.split * args.split_stride + (size_t)(ti.row0 + n) * args.ld_out + ch] =
+              __uint_as_float(v[j]);
+        }
+      }
+    }
+    release_tmem();
+  }
+}
+
 template <int KIND, int EPI, int BN_MAX, int STAGES, bool WN = false>
 __global__ void __launch_bounds__(384, 1)
     gemm_kernel(const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA,
@@ -570,8 +680,6 @@ __global__ void __launch_bounds__(384, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const int nchunks = ti.n_mma >> 4;
-      constexpr int CH = BN_MAX / 16;
       auto release_tmem = [&]() {
         tc_fence_before();
         __syncwarp();
@@ -668,105 +776,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; i < 16; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
-      } else if constexpr (EpiTraits<EPI>::glu) {
-        // a = glu(g, u) for this warp's chunks (c = sub + 2 i) straight out of TMEM;
-        // TMEM goes back to the MMA warp before the quantisation and stores.
-        constexpr int CH2 = (CH + 1) / 2;   // this warp's chunks: c = sub + 2 i
-        float a[CH2][16];
-#pragma unroll
-        for (int i = 0; i < CH2; ++i) {
-          const int c = sub + 2 * i;
-          if (c < nchunks) {
-            uint32_t g[16], u[16];
-            tmem_ld16(lane_base + c * 16, g);
-            tmem_ld16(lane_base + BN_MAX + c * 16, u);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) a[i][j] = glu_f<EpiTraits<EPI>::act>(__uint_as_float(g[j]), __uint_as_float(u[j]));
-          }
-        }
-        release_tmem();
-        const int ch = ti.mt * 128 + q * 32 + lane;  // intermediate channel
-#pragma unroll
-        for (int i = 0; i < CH2; ++i) {
-          const int c = sub + 2 * i;
-          if (c >= nchunks) break;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c * 16 + j;
-            if (n >= ti.n_valid) break;
-            const size_t row = (size_t)(ti.row0 + n);
-            if constexpr (EpiTraits<EPI>::mx8_out) {
-              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(a[i][j]) & 0x7FFFFFFFu);
-              const int e = mx_exp_e4m3(amax);
-              const float qv = a[i][j] * __uint_as_float((uint32_t)(127 - e) << 23);
-              const uint32_t code = f32x2_to_e4m3x2(qv, 0.0f) & 0xFFu;
-              ((uint8_t*)args.out0)[row * args.ld_out + ch] = (uint8_t)code;
-              if (lane == 0)   // scale byte for the down GEMM: K tile mt, block q, tile-major
-                ((uint8_t*)args.out1)[((size_t)ti.gt * args.m_tiles + ti.mt) * SF_TILE_BYTES +
-                                      sf_atom_offset(n) + q] = (uint8_t)(e + 127);
-            } else {
-              ((__nv_bfloat16*)args.out0)[row * args.ld_out + ch] = __float2bfloat16_rn(a[i][j]);
-            }
-          }
-        }
-      } else if constexpr (EPI == EPI_BF16) {
-        // round to bf16 pairs while draining TMEM, release it, then store
-        const int h = sub;
-        const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
-        uint32_t v[CH][8];
-        if (half_ok) {
-#pragma unroll
-          for (int c = 0; c < CH; ++c)
-            if (c < nchunks) {
-              uint32_t r[16];
-              tmem_ld16(lane_base + h * BN_MAX + c * 16, r);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const __nv_bfloat162 p2 =
-                    __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                v[c][j] = *(const uint32_t*)&p2;
-              }
-            }
-        }
-        release_tmem();
-        const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
-        if (half_ok && ch < args.M_total) {
-          uint16_t* out = (uint16_t*)args.out0;
-#pragma unroll
-          for (int c = 0; c < CH; ++c) {
-            if (c >= nchunks) break;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = c * 16 + j;
-              if (n >= ti.n_valid) break;
-              out[(size_t)(ti.row0 + n) * args.ld_out + ch] = (uint16_t)(v[c][j >> 1] >> ((j & 1) * 16));
-            }
-          }
-        }
       } else {
-        // fp32 results: store straight from TMEM chunk by chunk, release at the end
-        const int h = sub;
-        const int ch = ti.mt * 256 + h * 128 + q * 32 + lane;  // output channel
-        const bool half_ok = ti.mt * 256 + h * 128 < args.M_total;
-        if (half_ok) {
-          const bool ch_ok = ch < args.M_total;
-          for (int c = 0; c < nchunks; ++c) {
-            uint32_t v[16];
-            tmem_ld16(lane_base + h * BN_MAX + c * 16, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int n = c * 16 + j;
-              if (n >= ti.n_valid) break;
-              if (!ch_ok) continue;
-              ((float*)args.out0)[(size_t)ti.split * args.split_stride + (size_t)(ti.row0 + n) * args.ld_out + ch] =
-                  __uint_as_float(v[j]);
-            }
-          }
-        }
-        release_tmem();
+        epilogue_swapab<KIND, EPI, BN_MAX>(args, ti, lane_base, q, sub, lane, release_tmem);
       }
       acc_phase ^= 1;
 

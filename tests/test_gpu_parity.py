@@ -155,7 +155,7 @@ def _stage_checks(case, idx, w):
     xq_ref, xs_ref = mx.quantize_mx(x, "e4m3")
     xq = case.plan.debug_tensor(0, torch.uint8, (A, wl.d)).cpu().numpy()
     bn = api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_TILE_N)
-    assert bn in (32, 128, 176)
+    assert bn in (32, 128, 160, 176)
     ptr, nbytes = api.moe_debug_buffer(case.plan.handle, 1)
     xs = decode_tile_major_scales(case.plan.debug_tensor(1, torch.uint8, (nbytes,)).cpu().numpy(),
                                   counts, wl.d // 128, bn)
@@ -238,6 +238,29 @@ def test_layer_tile_configs_agree():
     api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 0)
     with pytest.raises(api.MoeError):
         api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 64)
+
+
+def test_layer_cta_pair_config_agrees():
+    """The CTA-pair routed GEMM (MOE_OPT_TILE_N = 160: clusters of two CTAs, M=256 MMAs
+    over both CTAs' weight rows, the token tile split between them) on a layer with even
+    m-tile counts (2I = 512 and d = 512: two 256-row m-tiles each).  Hot experts carry 400
+    rows, split into tiles of 144, 144 and 112 rows (MMA N 160, 160, 128); the others a few
+    rows (MMA N 32).  The result matches the oracle with the stage checks, and equals the
+    single-CTA 176-row configuration byte for byte: each output's K loop runs in the same
+    order."""
+    wl = synth.custom(seed=25, T=400, d=512, E=16, k=4, I=256, I_shared=128)
+    bias = torch.zeros(16)
+    bias[[2, 4, 9, 13]] = 40.0
+    case = Case(wl, bias=bias)
+    outs = []
+    for bn in (176, 160):
+        api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, bn)
+        _check_layer(case, stage_checks=True)
+        assert api.moe_plan_get_option(case.plan.handle, api.MOE_OPT_TILE_N) == bn
+        idx, w = case.plan.route(case.x, case.W_r, case.bias)
+        outs.append(case.plan.forward(case.x, idx, w, case.experts, case.shared).cpu())
+    assert torch.equal(outs[0], outs[1])
+    api.moe_plan_set_option(case.plan.handle, api.MOE_OPT_TILE_N, 0)
 
 
 def test_route_select_only_bias():
