@@ -614,20 +614,22 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         };
-        // Two K tiles per round: both stages' barriers are checked back to back and their 16
-        // MMAs issued in one run.  Each mbarrier wait costs the issuing thread about as much
-        // as one or two MMAs even when the stage has long landed, so pairing halves that
-        // overhead per MMA.  Each stage is still released as soon as its own MMAs commit.
-        for (int kt = ti.kb; kt < ti.ke; kt += 2) {
-          const bool two = kt + 1 < ti.ke;
+        // One or two K tiles per round: after the blocking wait for this stage, the next
+        // stage's barrier is tested once without waiting; if it has landed too, both
+        // stages' 16 MMAs are issued in one run.  Each mbarrier wait costs the issuing
+        // thread about as much as one or two MMAs, so pairing landed stages halves that
+        // overhead, while a stage is never held back waiting for its successor to land
+        // (which would keep its slot, and the loads it could make room for, waiting).
+        // Each stage is released as soon as its own MMAs commit.
+        for (int kt = ti.kb; kt < ti.ke;) {
+          const int kt0 = kt;
           const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
           ok = mbar_wait(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (ok) ++nfill;
-          if (ok && two) {
-            ok = mbar_wait(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
-            if (ok) ++nfill;
-          }
+          const bool two = ok && kt + 1 < ti.ke && mbar_try_wait(smem_u32(full_bar + stage2), phase2);
+          if (two) ++nfill;
+          kt += two ? 2 : 1;
           if (!ok) break;
           if (first) {
             // Everything the MMAs of a stage need except the stage offset is fixed per
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(384, 1)
             first = false;
           }
           tc_fence_after();
-          issue_stage(stage, kt > ti.kb ? 1u : 0u);
+          issue_stage(stage, kt0 > ti.kb ? 1u : 0u);
           tc_commit(smem_u32(empty_bar + stage));
           if (two) {
             issue_stage(stage2, 1u);

@@ -282,17 +282,17 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         };
-        // two K tiles per round, as in gemm_kernel; each stage released to both CTAs
-        for (int kt = kb; kt < ke; kt += 2) {
-          const bool two = kt + 1 < ke;
+        // one or two K tiles per round, as in gemm_kernel (the second only if it has
+        // already landed); each stage released to both CTAs
+        for (int kt = kb; kt < ke;) {
+          const int kt0 = kt;
           const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
           const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
           ok = mbar_wait_cluster(smem_u32(full_bar + stage), phase, args.status, abort_flag);
           if (ok) ++nfill;
-          if (ok && two) {
-            ok = mbar_wait_cluster(smem_u32(full_bar + stage2), phase2, args.status, abort_flag);
-            if (ok) ++nfill;
-          }
+          const bool two = ok && kt + 1 < ke && mbar_try_wait_cluster(smem_u32(full_bar + stage2), phase2);
+          if (two) ++nfill;
+          kt += two ? 2 : 1;
           if (!ok) break;
           if (first) {
             const int n_mma = stage_n[stage];
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(384, 1)
             first = false;
           }
           tc_fence_after();
-          issue_stage(stage, kt > kb ? 1u : 0u);
+          issue_stage(stage, kt0 > kb ? 1u : 0u);
           tc_commit2_mc(smem_u32(empty_bar + stage), 0x3);
           if (two) {
             issue_stage(stage2, 1u);
