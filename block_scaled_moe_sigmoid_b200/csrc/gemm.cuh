@@ -108,9 +108,13 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = CTRL_OFFSET + 1024 /*barriers*/ + 1024 /*align*/;
   // scale factors in TMEM, one 16-column buffer per pipeline stage:
   //   weights: 4 columns per 128-row half (+0, +4), tokens: 4 columns per 128 rows (+8, +12)
-  // after the accumulator (two halves of BN_MAX columns, or WN: 256 columns)
-  static constexpr int TMEM_SF = WN ? 256 : 2 * BN_MAX;
+  // after the accumulator buffers (each two halves of BN_MAX columns, or WN: 256 columns)
   static constexpr int TMEM_COLS = 512;
+  // Two accumulator buffers where TMEM holds them next to the scale buffers (the 32-row
+  // configuration): the MMAs of a tile then run while the epilogue drains the previous one.
+  static constexpr int ACC_BUFS = !WN && 4 * BN_MAX + 16 * STAGES <= TMEM_COLS ? 2 : 1;
+  static constexpr int ACC_COLS = 2 * BN_MAX;
+  static constexpr int TMEM_SF = WN ? 256 : ACC_BUFS * ACC_COLS;
   static constexpr int NUM_THREADS = 384;
   static_assert(BN_MAX % 16 == 0 && BN_MAX <= 256, "BN_MAX");
   static_assert(SFB_ATOMS <= 2, "scale buffer holds two B atoms");
@@ -364,9 +368,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* full_bar = (uint64_t*)ctrl;
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* sf_full = empty_bar + STAGES;        // scale blocks of the stage are in smem
-  uint64_t* acc_full = sf_full + STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain_bar = acc_empty + 1;
+  uint64_t* acc_full = sf_full + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* drain_bar = acc_empty + 2;
   uint64_t* drain_sf = drain_bar + 1;
   uint32_t* tmem_holder = (uint32_t*)(drain_sf + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
@@ -389,8 +393,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(smem_u32(empty_bar + s), 1);
       mbar_init(smem_u32(sf_full + s), 2);   // weight-scale and token-scale copies
     }
-    mbar_init(smem_u32(acc_full), 1);
-    mbar_init(smem_u32(acc_empty), 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(acc_full + b), 1);
+      mbar_init(smem_u32(acc_empty + b), 8);
+    }
     mbar_init(smem_u32(drain_bar), 1);
     mbar_init(smem_u32(drain_sf), 1);
     *abort_flag = 0;
@@ -568,7 +574,8 @@ __global__ void __launch_bounds__(384, 1)
       // 128-byte-swizzled K-major descriptor of stage 0's A tile; other tiles are offsets
       const uint64_t desc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0;
+      int tcount = 0;
       bool ok = true;
       int nfill = 0;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -585,6 +592,9 @@ __global__ void __launch_bounds__(384, 1)
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
         uint32_t idesc[4];
         bool first = true;
+        const int abuf = tcount % C::ACC_BUFS;
+        const uint32_t acc_phase = (uint32_t)(tcount / C::ACC_BUFS) & 1u;
+        const uint32_t acc_t = tmem_base + (uint32_t)(abuf * C::ACC_COLS);
         // the MMAs of the K tile held by smem stage st: 4 K-blocks x 2 halves (WN: 4 K-blocks)
         auto issue_stage = [&](int st, uint32_t acc0) {
           const uint64_t a_desc = desc0 + (uint64_t)((st * C::STAGE_BYTES) >> 4);
@@ -594,7 +604,7 @@ __global__ void __launch_bounds__(384, 1)
             // token tile (A, M=128) x all 256 weight rows (B, N=256), one MMA per K block
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              mma_mxf8f6f4(tmem_base, b_desc + (uint64_t)((32 * j) >> 4), a_desc + (uint64_t)((32 * j) >> 4), idesc[j],
+              mma_mxf8f6f4(acc_t, b_desc + (uint64_t)((32 * j) >> 4), a_desc + (uint64_t)((32 * j) >> 4), idesc[j],
                            (tsf + 8) | ((uint32_t)j << 30), tsf | ((uint32_t)j << 30), j > 0 ? 1u : acc0);
           } else {
 #pragma unroll
@@ -606,10 +616,10 @@ __global__ void __launch_bounds__(384, 1)
                 const uint64_t bdesc = b_desc + (uint64_t)((32 * j) >> 4);
                 const uint32_t acc = j > 0 ? 1u : acc0;
                 if constexpr (KIND == KIND_MX)
-                  mma_mxf8f6f4(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], (tsf + 4 * h) | ((uint32_t)j << 30),
+                  mma_mxf8f6f4(acc_t + h * BN_MAX, adesc, bdesc, idesc[j], (tsf + 4 * h) | ((uint32_t)j << 30),
                                (tsf + 8) | ((uint32_t)j << 30), acc);
                 else
-                  mma_bf16(tmem_base + h * BN_MAX, adesc, bdesc, idesc[j], acc);
+                  mma_bf16(acc_t + h * BN_MAX, adesc, bdesc, idesc[j], acc);
               }
             }
           }
@@ -641,7 +651,7 @@ __global__ void __launch_bounds__(384, 1)
               idesc[j] = WN ? idesc_mx_e4m3_e2m1(128, 256, j, j)
                             : (KIND == KIND_MX ? idesc_mx_e2m1_e4m3(128, n_mma, j, j) : idesc_bf16(128, n_mma));
             // the accumulator is free once the epilogue has drained the previous tile
-            ok = mbar_wait(smem_u32(acc_empty), acc_phase ^ 1, args.status, abort_flag);
+            ok = mbar_wait(smem_u32(acc_empty + abuf), acc_phase ^ 1, args.status, abort_flag);
             if (!ok) break;
             first = false;
           }
@@ -659,8 +669,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(acc_full));
-        acc_phase ^= 1;
+        tc_commit(smem_u32(acc_full + abuf));
+        ++tcount;
       }
       // make sure every MMA this thread issued has finished before TMEM is released
       tc_commit(smem_u32(drain_bar));
@@ -672,20 +682,23 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int sub = (warp - 2) >> 2;   // 0 or 1
-    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-    uint32_t acc_phase = 0;
+    const uint32_t lane_base0 = tmem_base + ((uint32_t)(q * 32) << 16);
+    int tcount = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       TileInfo ti;
       gemm_decode_tile(args, BN_MAX, t, ti);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(smem_u32(acc_full), acc_phase, args.status, abort_flag);
+      const int abuf = tcount % C::ACC_BUFS;
+      const uint32_t acc_phase = (uint32_t)(tcount / C::ACC_BUFS) & 1u;
+      const uint32_t lane_base = lane_base0 + (uint32_t)(abuf * C::ACC_COLS);
+      if (lane == 0) ok = mbar_wait(smem_u32(acc_full + abuf), acc_phase, args.status, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
       auto release_tmem = [&]() {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+        if (lane == 0) mbar_arrive(smem_u32(acc_empty + abuf));
       };
       if constexpr (WN) {
         // TMEM lane = token row of the tile (quarter q: rows 32q..32q+31), column = weight
@@ -781,7 +794,7 @@ __global__ void __launch_bounds__(384, 1)
       } else {
         epilogue_swapab<KIND, EPI, BN_MAX>(args, ti, lane_base, q, sub, lane, release_tmem);
       }
-      acc_phase ^= 1;
+      ++tcount;
 
     }
   }
