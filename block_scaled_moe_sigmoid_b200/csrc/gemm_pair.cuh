@@ -9,12 +9,18 @@
 // its 256 weight rows but only half the token rows per stage: 42 KB instead of 54 KB of
 // tiles for the same tensor work, which fits five stages instead of four.  The routed GEMM
 // is bound by the bytes its stage ring holds in flight, so the extra stage is the point.
+// Measured on the Kimi-K3 prefill shapes, it is nonetheless slower than gemm_kernel's
+// single-CTA tiles (each stage now waits for both SMs' loads), so it runs only when the
+// 160-row tile configuration is selected explicitly.  Its outputs are bit-identical to the
+// single-CTA kernel's: the fp32 accumulation order over K is the same.
 //
 // Roles per CTA (384 threads), rank 0 = leader, rank 1 = peer:
 //   warp 0   weight rows of its own m-tile (TMA .cta_group::2: the completed bytes count on
 //            the leader's full barrier) and their scale atoms (bulk copy, local barrier);
+//            the leader's also arms its full barrier with both CTAs' weight bytes;
 //   warp 10  its half of the token rows (TMA .cta_group::2, leader's barrier) and the whole
-//            tile's token scale atoms (bulk copy, local barrier);
+//            tile's token scale atoms (bulk copy, local barrier); the leader's also arms
+//            its full barrier with the whole tile's token bytes;
 //   warp 11  leader: once both CTAs' scale atoms of a stage are in shared memory (the peer
 //            forwards its local completion with a remote arrive), copies them into both
 //            CTAs' TMEM (tcgen05.cp .cta_group::2) and commits to the stage's full barrier;
@@ -25,8 +31,11 @@
 //   warps 2..9  the swap-AB epilogue on the CTA's own TMEM rows; the accumulator is free
 //            again when all 16 epilogue warps of the pair have arrived on the leader's
 //            acc_empty.
-// Producers arm the leader's full barrier with their own bytes (the peer's arrivals are
-// remote), so a stage is full when both CTAs' tiles and the leader's scale copies are done.
+// Only the leader's producers arrive on its full barrier, each expecting both CTAs' bytes;
+// the peer's copies only complete bytes on it (no remote arrivals, which measured 15-18%
+// slower).  A stage is full when both CTAs' tiles and the leader's scale copies are done;
+// the peer arms nothing before its own empty barrier has released the stage, so its bytes
+// always land in the phase the leader is arming.
 #pragma once
 #include "gemm.cuh"
 
@@ -91,7 +100,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* drain_sf = drain_bar + 1;
   uint32_t* tmem_holder = (uint32_t*)(drain_sf + 1);
   volatile int* abort_flag = (volatile int*)(tmem_holder + 1);
-  // Abort cleanup counters: [0] weight producer, [1] token producer (stages armed),
+  // Abort cleanup counters: [0] weight producer, [1] token producer (stages issued; the
+  // leader's also armed them),
   // [2] leader scale warp (stages committed), [3] leader MMA (full phases consumed),
   // [4] scale warp (sf_full phases consumed).
   int* fills = (int*)(tmem_holder + 2);
@@ -104,8 +114,9 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // weight + token producers of both CTAs, plus the leader's scale-copy commit
-      mbar_init(smem_u32(full_bar + s), 5);
+      // the leader's weight and token producers (each arming both CTAs' bytes), plus the
+      // leader's scale-copy commit
+      mbar_init(smem_u32(full_bar + s), 3);
       mbar_init(smem_u32(empty_bar + s), 1);
       mbar_init(smem_u32(sf_full + s), 2);
       mbar_init(smem_u32(sf_peer + s), 1);
@@ -159,7 +170,7 @@ __global__ void __launch_bounds__(384, 1)
                 "l"(args.sfa + blk * 1024), "r"(sb)
                 : "memory");
             const uint32_t fb = leader_addr(full_bar + stage);
-            mbar_arrive_expect_tx_cluster(fb, C::A_TX);
+            if (leader) mbar_arrive_expect_tx(smem_u32(full_bar + stage), 2 * C::A_TX);
             tma_load_2d_pair(smem_u32(smem + stage * C::STAGE_BYTES), &tmA, fb, 0, (int)(blk * C::BM), pol_a);
           }
         }
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(384, 1)
               "l"(args.sfb + ((size_t)ti.gt * args.k_tiles + kt) * SF_TILE_BYTES), "r"(sfb_bytes), "r"(sb)
               : "memory");
           const uint32_t fb = leader_addr(full_bar + stage);
-          mbar_arrive_expect_tx_cluster(fb, half * 128);
+          if (leader) mbar_arrive_expect_tx(smem_u32(full_bar + stage), ti.n_mma * 128);
           tma_load_2d_pair(smem_u32(smem + stage * C::STAGE_BYTES + C::A_BYTES), &tmB.box[nB - 1], fb,
                            (kt % args.kb_wrap) * C::BK, ti.row0 + rank * half, pol_b);
         }
@@ -357,9 +368,8 @@ __global__ void __launch_bounds__(384, 1)
     // flight into either CTA's shared memory land, supplying the arrivals of roles that
     // stopped early.  The leader's full ring counts both CTAs' producers.
     if (leader) {
-      const int arrived[5] = {fills[0], fills[1], (int)ld_shared_cluster_u32(mapa_shared(smem_u32(fills + 0), 1)),
-                              (int)ld_shared_cluster_u32(mapa_shared(smem_u32(fills + 1), 1)), fills[2]};
-      drain_ring(full_bar, STAGES, arrived, 5, fills[3]);
+      const int arrived[3] = {fills[0], fills[1], fills[2]};
+      drain_ring(full_bar, STAGES, arrived, 3, fills[3]);
     }
     drain_ring(sf_full, STAGES, fills, 2, fills[4]);
   }
