@@ -18,6 +18,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -30,14 +31,15 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s at K3 shape (T=8192); % FP4 tensor peak, decode % HBM BW"
 UNIT = "tokens/s"
 
-# The GEMM sources whose hash keys a recorded DRAM-traffic figure.
+# The GEMM sources whose hash (over their code, comments dropped) keys a recorded
+# DRAM-traffic figure.
 GEMM_SOURCES = ("gemm.cuh", "ptx.cuh", "tiling.cuh")
 # DRAM bytes (read + write) of one launch of the routed gate/up GEMM, from an ncu capture
 # (`--metrics dram__bytes_read.sum,dram__bytes_write.sum`, one pass) of the kernel built
 # from the GEMM sources with the given hash.  A figure whose hash no longer matches the
 # sources is not reported.
 GATE_UP_TRAFFIC = {
-    ("k3_prefill_t8192", 8192): {"bytes": 22092875264 + 408987392, "sha16": "1f4291fbf38aa5b4",
+    ("k3_prefill_t8192", 8192): {"bytes": 22092875264 + 408987392, "sha16": "a78528257fadb9ff",
                                   "how": "timed-step launch of the full T=8192 workload"},
 }
 
@@ -223,12 +225,20 @@ def setup(wl, T, device):
     return x, W_r, bias, plan, ex, sh
 
 
+_C_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def source_sha16(*names):
-    """First 16 hex digits of the sha256 of the named CUDA sources of the package."""
+    """First 16 hex digits of the sha256 of the named CUDA sources of the package, taken
+    over their code only: comments, trailing blanks and empty lines are dropped, so that a
+    recorded figure follows the kernels and not the wording of their comments."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "block_scaled_moe_sigmoid_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "block_scaled_moe_sigmoid_b200", "csrc", n), encoding="utf-8") as f:
+            code = _C_COMMENT.sub("", f.read())
+        lines = [ln.rstrip() for ln in code.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
+        h.update(b"\0")
     return h.hexdigest()[:16]
 
 

@@ -24,7 +24,7 @@
 // Roles (384 threads): warp 0 loads the weight tiles (TMA, plus a bulk copy of their
 // scales), warp 10 loads the token rows (one TMA box, plus a bulk copy of their scales),
 // warp 11 copies each stage's scale factors into TMEM (KIND_MX), warp 1 owns TMEM and one
-// lane issues the MMAs, two K tiles per round, warps 2..9 run the epilogue (lane quarter =
+// lane issues the MMAs, one or two K tiles per round, warps 2..9 run the epilogue (lane quarter =
 // warp % 4).  The producers and the scale warp complete the same stage independently.
 //
 // Orientation WN (KIND_MX, a few tokens per expert): the token rows are the MMA's M side
@@ -592,6 +592,7 @@ __global__ void __launch_bounds__(384, 1)
         const bool h1 = ti.mt * C::BM + 128 < args.M_total;
         uint32_t idesc[4];
         bool first = true;
+        // this CTA's tile count picks the accumulator buffer and its barrier phase
         const int abuf = tcount % C::ACC_BUFS;
         const uint32_t acc_phase = (uint32_t)(tcount / C::ACC_BUFS) & 1u;
         const uint32_t acc_t = tmem_base + (uint32_t)(abuf * C::ACC_COLS);
@@ -650,7 +651,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 4; ++j)
               idesc[j] = WN ? idesc_mx_e4m3_e2m1(128, 256, j, j)
                             : (KIND == KIND_MX ? idesc_mx_e2m1_e4m3(128, n_mma, j, j) : idesc_bf16(128, n_mma));
-            // the accumulator is free once the epilogue has drained the previous tile
+            // the accumulator buffer is free once the epilogue has drained the tile that
+            // last used it (the previous tile, or the one before with two buffers)
             ok = mbar_wait(smem_u32(acc_empty + abuf), acc_phase ^ 1, args.status, abort_flag);
             if (!ok) break;
             first = false;

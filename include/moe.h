@@ -283,15 +283,18 @@ moe_status_t moe_pack_shared_bf16(int d, int I_shared, const void* w_gate, const
  *   32 rows (6-stage pipeline) when T*k <= 8*E, i.e. a few tokens per expert and a pure
  *   weight stream, else 176 rows (4 stages); both put 256 weight rows on the MMA's M side
  *   and the token rows on its N side.  128 selects the other orientation: token rows on M
- *   (up to 128 per tile) and 256 weight rows on N.  32, 128 or 176 forces one
- *   configuration; any other value is MOE_ERR_INVALID_ARG.  The dense shared-expert GEMMs
- *   use 32-row tiles when T*k <= 8*E and 176 otherwise.  The K loop runs in the same order
- *   in all three, and the tensor core accumulates a row the same way in either
- *   orientation: results are identical.
+ *   (up to 128 per tile) and 256 weight rows on N.  160 selects tiles of up to 160 token
+ *   rows run on clusters of two CTAs (one MMA spans two SMs: each holds its own 256 weight
+ *   rows and half of the token rows; five pipeline stages); a GEMM whose weight rows do not
+ *   form an even number of 256-row tiles runs its 160-row tiles on single CTAs instead.
+ *   32, 128, 160 or 176 forces one configuration; any other value is MOE_ERR_INVALID_ARG.
+ *   The dense shared-expert GEMMs use 32-row tiles when T*k <= 8*E and 176 otherwise.  The
+ *   K loop runs in the same order in all of them, and the tensor core accumulates a row the
+ *   same way in either orientation and on one or two SMs: results are identical.
  * MOE_OPT_ROUTER_SPLIT (read only): the number of K splits the last moe_route used for
  *   the router GEMM (1 = none).  With few tokens the router splits d over up to one
- *   CTA per SM; the CTA that finishes a tile's last split adds the fp32 partials in split
- *   order (plus the bias) inside the same kernel.
+ *   CTA per SM; each split stores its fp32 partial, and the selection kernel that follows
+ *   adds the partials in split order (plus the bias) before it selects.
  * MOE_OPT_SHARED_SPLIT / MOE_OPT_SHARED_SPLIT_DOWN (read only): K splits of the shared
  *   expert's gate/up and down GEMMs in the last moe_forward (1 = none; 0 without a shared
  *   expert).  With few tokens these dense GEMMs split K over the SMs.  Each split GEMM writes
@@ -313,8 +316,8 @@ moe_status_t moe_plan_get_option(moe_plan_t plan, int option, int* value);
  * n >= MOE_NUM_STAGES entries; `launches` may be NULL), then forgets them. */
 enum {
   MOE_STAGE_ROUTER_SPLIT = 0,    /* W_r -> three bf16 planes */
-  MOE_STAGE_ROUTER_GEMM = 1,     /* logits on the tensor cores + fused sigmoid top-k */
-  MOE_STAGE_TOPK = 2,            /* (sigmoid top-k is fused into the router kernel: unused) */
+  MOE_STAGE_ROUTER_GEMM = 1,     /* logits on the tensor cores (fp32 partials when K is split) */
+  MOE_STAGE_TOPK = 2,            /* split sum + bias, top-k selection, sigmoid weights */
   MOE_STAGE_PERMUTE = 3,         /* histogram, scan, placement (3 kernels) */
   MOE_STAGE_QUANT = 4,           /* MXFP8 quantise + scatter to expert order */
   MOE_STAGE_GATE_UP = 5,         /* routed gate/up GEMM + GLU + MXFP8 requant */
