@@ -228,13 +228,15 @@ def setup(wl, T, device):
 _C_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
 
 
-def source_sha16(*names):
-    """First 16 hex digits of the sha256 of the named CUDA sources of the package, taken
-    over their code only: comments, trailing blanks and empty lines are dropped, so that a
-    recorded figure follows the kernels and not the wording of their comments."""
+def source_sha16(*names, csrc=None):
+    """First 16 hex digits of the sha256 of the named CUDA sources of the package (or of
+    the directory `csrc`), taken over their code only: comments, trailing blanks and empty
+    lines are dropped, so that a recorded figure follows the kernels and not the wording of
+    their comments."""
+    csrc = csrc or os.path.join(ROOT, "block_scaled_moe_sigmoid_b200", "csrc")
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "block_scaled_moe_sigmoid_b200", "csrc", n), encoding="utf-8") as f:
+        with open(os.path.join(csrc, n), encoding="utf-8") as f:
             code = _C_COMMENT.sub("", f.read())
         lines = [ln.rstrip() for ln in code.splitlines()]
         h.update("\n".join(ln for ln in lines if ln).encode())
