@@ -7,8 +7,10 @@
 // token tile, whose first N/2 rows sit in the even CTA's shared memory and the rest in the
 // odd CTA's) x K=32, and each CTA's TMEM receives its own 128 rows x N.  So each SM holds
 // its 256 weight rows but only half the token rows per stage: 42 KB instead of 54 KB of
-// tiles for the same tensor work, which fits five stages instead of four.  The routed GEMM
-// is bound by the bytes its stage ring holds in flight, so the extra stage is the point.
+// tiles for the same tensor work (five stages instead of four), and each SM fetches only
+// half of each token tile from L2.  The single-CTA routed GEMM moves about as many bytes
+// from L2 into shared memory as the GPU delivers to TMA loads on all SMs, and the token
+// rows, re-read by every m-tile, are half of them: halving those is the point.
 // Measured on the Kimi-K3 prefill shapes, it is nonetheless slower than gemm_kernel's
 // single-CTA tiles (each stage now waits for both SMs' loads), so it runs only when the
 // 160-row tile configuration is selected explicitly.  Its outputs are bit-identical to the
