@@ -49,3 +49,12 @@ def test_recorded_traffic_entries_are_well_formed():
         assert isinstance(workload, str) and T > 0
         assert rec["bytes"] > 0 and len(rec["sha16"]) == 16
         int(rec["sha16"], 16)
+
+
+def test_prefill_traffic_record_is_keyed_on_the_current_gemm_sources():
+    # the recorded figure is reported only while the GEMM code it was captured on is unchanged
+    rec = bench.traffic_record("k3_prefill_t8192", 8192)
+    key = bench.source_sha16(*bench.GEMM_SOURCES)
+    stored = bench.GATE_UP_TRAFFIC[("k3_prefill_t8192", 8192)]["sha16"]
+    assert (rec is not None) == (key == stored)
+    assert bench.traffic_record("k3_decode_t64", 64) is None
