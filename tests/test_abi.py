@@ -64,6 +64,12 @@ def test_host_side_argument_checks_without_gpu():
         assert L.moe_plan_get_option(h, opt, ctypes.byref(v)) == 0
     assert L.moe_plan_get_option(h, 99, ctypes.byref(v)) == 1
     assert L.moe_plan_set_option(h, 3, 1) == 1                          # read-only option
+    for tile_n in (0, 32, 128, 160, 176):                               # the tile configurations
+        assert L.moe_plan_set_option(h, 2, tile_n) == 0
+    for tile_n in (-1, 16, 64, 96, 192, 256):
+        assert L.moe_plan_set_option(h, 2, tile_n) == 1
+    assert L.moe_plan_set_option(h, 0, 65) == 1                         # prefetch distance <= 64
+    assert L.moe_plan_set_option(h, 0, 8) == 0 and L.moe_plan_set_option(h, 0, 0) == 0
     assert L.moe_plan_destroy(h) == 0
     assert L.moe_quant_mxfp8(None, 4, 33, None, None, None) == 2
     assert L.moe_status_string(3) == b"misaligned pointer"
